@@ -1,0 +1,416 @@
+"""Pins for the fp64 oracle: each test ties one oracle routine to something other
+than itself -- a hand-worked example, a closed form, an invariant, brute force
+with Python complex numbers, or exact rational arithmetic.  CPU only."""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle as O
+from conftest import read_golden
+
+
+# ---------------------------------------------------------------------------
+# Phase rule
+# ---------------------------------------------------------------------------
+def _grid_points():
+    """fp32 grid: integer lattice -4..4, diagonal neighbours at many magnitudes,
+    subnormals and signed zeros (as float64 arrays of fp32 values)."""
+    pts = []
+    ints = np.arange(-4, 5, dtype=np.float32)
+    for a in ints:
+        for b in ints:
+            pts.append((a, b))
+    mags = np.array([1.4e-45, 1e-40, 1.17549435e-38, 1e-30, 1e-3, 0.02, 1.0, 3.7, 1e20, 3e38], np.float32)
+    for m in mags:
+        up = np.nextafter(m, np.float32(np.inf))
+        dn = np.nextafter(m, np.float32(0))
+        for s1 in (1, -1):
+            for s2 in (1, -1):
+                for (u, v) in ((m, m), (m, up), (up, m), (m, dn), (dn, m)):
+                    pts.append((np.float32(s1 * u), np.float32(s2 * v)))
+    for z1 in (0.0, -0.0):
+        for z2 in (0.0, -0.0, 1.0, -1.0, 1e-45, -1e-45):
+            pts.append((np.float32(z1), np.float32(z2)))
+            pts.append((np.float32(z2), np.float32(z1)))
+    a = np.array([p[0] for p in pts], np.float32).astype(np.float64)
+    b = np.array([p[1] for p in pts], np.float32).astype(np.float64)
+    return a, b
+
+
+def test_phase_rule_exact_form_matches_atan2_form_on_fp32_grid():
+    a, b = _grid_points()
+    assert a.size > 300
+    np.testing.assert_array_equal(O.phase_code(a, b), O.phase_code_atan2(a, b))
+
+
+def test_phase_rule_exact_form_matches_atan2_form_on_random_fp32():
+    rng = np.random.default_rng(123)
+    a = rng.standard_normal(200000).astype(np.float32).astype(np.float64)
+    b = rng.standard_normal(200000).astype(np.float32).astype(np.float64)
+    np.testing.assert_array_equal(O.phase_code(a, b), O.phase_code_atan2(a, b))
+
+
+def test_phase_rule_hand_sector_table():
+    rows = read_golden("phase_rule_sectors.txt")
+    a = np.array([float(r[0]) for r in rows])
+    b = np.array([float(r[1]) for r in rows])
+    want = np.array([int(r[2]) for r in rows], np.uint8)
+    np.testing.assert_array_equal(O.phase_code(a, b), want)
+    np.testing.assert_array_equal(O.phase_code_atan2(a, b), want)
+
+
+def test_phase_rule_matches_nearest_codeword_off_ties():
+    """Away from ties the rule picks the codeword nearest to w/|w| (brute force over 4 entries)."""
+    rng = np.random.default_rng(7)
+    w = rng.standard_normal(5000) + 1j * rng.standard_normal(5000)
+    u = w / np.abs(w)
+    dist = np.abs(u[:, None] - np.array(O.CODEBOOK)[None, :])
+    want = np.argmin(dist, axis=1).astype(np.uint8)
+    np.testing.assert_array_equal(O.phase_code(w.real, w.imag), want)
+
+
+def test_phase_rule_rotation_equivariance():
+    """k(i w) = k(w) + 1 and k(-w) = k(w) + 2 (mod 4) for w != 0; i w = -b + i a is exact."""
+    a, b = _grid_points()
+    rng = np.random.default_rng(11)
+    a = np.concatenate([a, rng.standard_normal(5000)])
+    b = np.concatenate([b, rng.standard_normal(5000)])
+    nz = ~((a == 0) & (b == 0))
+    a, b = a[nz], b[nz]
+    k = O.phase_code(a, b).astype(np.int64)
+    np.testing.assert_array_equal(O.phase_code(-b, a), (k + 1) % 4)
+    np.testing.assert_array_equal(O.phase_code(-a, -b), (k + 2) % 4)
+
+
+def test_times_i_is_swap_and_negate():
+    """("iFairy talk notes" §2.3.1) i (a + ib) = -b + ia for every bf16 pair tried."""
+    rng = np.random.default_rng(5)
+    xr = O.bf16_round(rng.standard_normal(1000).astype(np.float32)).astype(np.float64)
+    xi = O.bf16_round(rng.standard_normal(1000).astype(np.float32)).astype(np.float64)
+    for r, i in zip(xr, xi):
+        z = 1j * complex(r, i)
+        assert z.real == -i and z.imag == r
+
+
+def test_codebook_br_bi():
+    br, bi = O.code_to_br_bi(np.arange(4, dtype=np.uint8))
+    for k in range(4):
+        assert complex(int(br[k]), int(bi[k])) == O.CODEBOOK[k]
+    # exactly one of Re, Im is zero for every codeword ("iFairy article" §二.1)
+    assert np.all((br == 0) ^ (bi == 0))
+
+
+# ---------------------------------------------------------------------------
+# Scales and residual stages
+# ---------------------------------------------------------------------------
+def test_two_stage_hand_example():
+    g = {r[0]: r[1:] for r in read_golden("two_stage_example.txt")}
+    w_re = np.array([float(v) for v in g["w_re"]], np.float32)[None, :]
+    w_im = np.array([float(v) for v in g["w_im"]], np.float32)[None, :]
+    packed, scales, _ = O.quantize_tensor(w_re, w_im, 2)
+    k = O.unpack_codes(packed[:, 0])
+    np.testing.assert_array_equal(k[0], [int(v) for v in g["k1"]])
+    np.testing.assert_array_equal(k[1], [int(v) for v in g["k2"]])
+    assert scales[0, 0] == np.float32(float(g["s1"][0]))
+    assert scales[0, 1] == np.float32(float(g["s1"][1]))
+    assert scales[1, 0] == np.float32(Fraction(17, 12))   # 4.25 / 3
+    assert scales[1, 1] == np.float32(float(g["s2"][1]))
+    assert list(packed[0, 0]) == [int(v, 16) for v in g["bytes1"]]
+    assert list(packed[1, 0]) == [int(v, 16) for v in g["bytes2"]]
+
+
+def _stage_python_loop(a, b):
+    """Element-by-element stage with Python floats and the atan2 form (independent route)."""
+    S = [0.0, 0.0]
+    C = [0, 0]
+    ks = []
+    for x, y in zip(a.ravel().tolist(), b.ravel().tolist()):
+        k = int(O.phase_code_atan2(np.array([x]), np.array([y]))[0])
+        ks.append(k)
+        if k % 2 == 0:
+            S[0] += abs(x)
+            C[0] += 1
+        else:
+            S[1] += abs(y)
+            C[1] += 1
+    return np.array(ks, np.uint8).reshape(a.shape), S, C
+
+
+def test_quantize_stage_matches_python_loop():
+    rng = np.random.default_rng(3)
+    a = (0.02 * rng.standard_normal((6, 16))).astype(np.float32).astype(np.float64)
+    b = (0.02 * rng.standard_normal((6, 16))).astype(np.float32).astype(np.float64)
+    k, (s_re, s_im), sums = O.quantize_stage(a, b)
+    k2, S, C = _stage_python_loop(a, b)
+    np.testing.assert_array_equal(k, k2)
+    assert sums[1] == C[0] and sums[3] == C[1]
+    assert abs(sums[0] - S[0]) <= 1e-15 * S[0] and abs(sums[2] - S[1]) <= 1e-15 * S[1]
+    assert s_re == np.float32(S[0] / C[0]) and s_im == np.float32(S[1] / C[1])
+
+
+def test_energy_identity_and_least_squares():
+    """||r_{t+1}||^2 = ||r_t||^2 - C_re s_re^2 - C_im s_im^2 when s is the class mean
+    (codes carry sign(Re r) on +-1 entries, sign(Im r) on +-i entries); any other scale is worse."""
+    rng = np.random.default_rng(9)
+    a = (0.02 * rng.standard_normal((64, 96))).astype(np.float32).astype(np.float64)
+    b = (0.02 * rng.standard_normal((64, 96))).astype(np.float32).astype(np.float64)
+    for _stage in range(3):
+        k, _, (S_re, C_re, S_im, C_im) = O.quantize_stage(a, b)
+        s_re, s_im = S_re / C_re, S_im / C_im
+        br, bi = O.code_to_br_bi(k)
+
+        def energy(sr, si):
+            return float(np.sum((a - sr * br) ** 2 + (b - si * bi) ** 2))
+
+        e0 = float(np.sum(a * a + b * b))
+        e1 = energy(s_re, s_im)
+        want = e0 - C_re * s_re ** 2 - C_im * s_im ** 2
+        assert abs(e1 - want) <= 1e-12 * e0
+        for eps in (1e-3, -1e-3):
+            assert energy(s_re * (1 + eps), s_im) > e1
+            assert energy(s_re, s_im * (1 + eps)) > e1
+        a, b = a - s_re * br, b - s_im * bi
+
+
+def test_real_only_weights_reduce_to_sign_binarisation():
+    """Im w = 0: codes are +-1 by sign(Re w), s_re = mean |w| (binary-weight rule), s_im = 0."""
+    rng = np.random.default_rng(4)
+    w = (0.02 * rng.standard_normal((8, 32))).astype(np.float32)
+    packed, scales, _ = O.quantize_tensor(w, np.zeros_like(w), 1)
+    k = O.unpack_codes(packed[0])
+    np.testing.assert_array_equal(k, np.where(w >= 0, 0, 2))
+    assert scales[0, 0] == np.float32(np.mean(np.abs(w.astype(np.float64))))
+    assert scales[0, 1] == 0.0
+
+
+def test_scales_swap_under_multiplication_by_i():
+    rng = np.random.default_rng(6)
+    a = (0.02 * rng.standard_normal((16, 64))).astype(np.float32)
+    b = (0.03 * rng.standard_normal((16, 64))).astype(np.float32)
+    p1, s1, _ = O.quantize_tensor(a, b, 2)
+    p2, s2, _ = O.quantize_tensor(-b, a, 2)     # i w
+    assert s1[0, 0] == s2[0, 1] and s1[0, 1] == s2[0, 0]
+    k1 = O.unpack_codes(p1[0]).astype(int)
+    k2 = O.unpack_codes(p2[0]).astype(int)
+    np.testing.assert_array_equal(k2, (k1 + 1) % 4)
+
+
+def test_isotropic_gaussian_codes_are_uniform():
+    """Isotropic weights use the four codewords equally (cf. "iFairy article" §四), within 5 sigma."""
+    rng = np.random.default_rng(0)
+    n = 400000
+    k = O.phase_code(rng.standard_normal(n), rng.standard_normal(n))
+    counts = np.bincount(k, minlength=4)
+    sigma = np.sqrt(n * 0.25 * 0.75)
+    assert np.all(np.abs(counts - n / 4) < 5 * sigma)
+
+
+def test_second_stage_is_rule_on_complex_residual():
+    """Stage 2 codes equal the rule applied to w - w_hat_1 formed with complex arithmetic."""
+    rng = np.random.default_rng(8)
+    wr = (0.02 * rng.standard_normal((12, 40))).astype(np.float32)
+    wi = (0.02 * rng.standard_normal((12, 40))).astype(np.float32)
+    packed, scales, _ = O.quantize_tensor(wr, wi, 2)
+    w_hat1 = O.dequantize(packed[:1], scales[:1])
+    r = (wr.astype(np.float64) + 1j * wi.astype(np.float64)) - w_hat1
+    np.testing.assert_array_equal(O.unpack_codes(packed[1]), O.phase_code(r.real, r.imag))
+
+
+def test_chunked_quantizer_matches_whole_tensor():
+    rng = np.random.default_rng(10)
+    wr = (0.02 * rng.standard_normal((37, 24))).astype(np.float32)
+    wi = (0.02 * rng.standard_normal((37, 24))).astype(np.float32)
+    p1, s1, _ = O.quantize_tensor(wr, wi, 3)
+    p2, s2, _ = O.quantize_tensor(wr, wi, 3, row_chunk=5)
+    np.testing.assert_array_equal(p1, p2)
+    np.testing.assert_allclose(s1, s2, rtol=1e-7)
+
+
+def test_nonfinite_weight_is_taken_as_zero():
+    wr = np.array([[np.nan, 1.0, -2.0, 0.5]], np.float32)
+    wi = np.array([[0.0, np.inf, 0.1, 3.0]], np.float32)
+    packed, scales, sums = O.quantize_tensor(wr, wi, 1)
+    k = O.unpack_codes(packed[0])[0]
+    assert list(k) == [0, 0, 2, 1]
+    S_re, C_re, S_im, C_im = sums[0]
+    assert (S_re, C_re, S_im, C_im) == (2.0, 3, 3.0, 1)
+
+
+def test_empty_class_gives_zero_scale():
+    wr = np.ones((2, 4), np.float32)
+    wi = np.zeros((2, 4), np.float32)
+    _, scales, _ = O.quantize_tensor(wr, wi, 2)
+    assert scales[0, 0] == 1.0 and scales[0, 1] == 0.0
+    # stage 2 residual is exactly zero everywhere -> all code 0, mean 0
+    assert scales[1, 0] == 0.0 and scales[1, 1] == 0.0
+
+
+def test_near_boundary_mask():
+    a = np.array([1.0, 1.0, 1.0, 1e-9, 0.5])
+    b = np.array([1.0, 1.0 + 1e-7, 0.9, 0.0, 0.1])
+    m = O.near_boundary_mask(a, b, prev_scale_sum=1.0)
+    assert list(m) == [True, True, False, True, False]
+
+
+# ---------------------------------------------------------------------------
+# Packing
+# ---------------------------------------------------------------------------
+def test_pack_hand_byte_and_round_trip():
+    assert O.pack_codes(np.array([0, 1, 2, 3], np.uint8))[0] == 0xE4   # 0b11_10_01_00
+    rng = np.random.default_rng(2)
+    k = rng.integers(0, 4, size=(5, 64), dtype=np.uint8)
+    np.testing.assert_array_equal(O.unpack_codes(O.pack_codes(k)), k)
+
+
+def test_storage_is_two_bits_per_weight():
+    """2 bits per complex weight: N K / 4 bytes per stage and branch; 1.3e9 weights ~ 325 MB
+    ("iFairy talk notes" Q&A quotes about 300 MB; "iFairy article" §一 quotes 1/8 of FP16)."""
+    k = np.zeros((48, 128), np.uint8)
+    assert O.pack_codes(k).nbytes == 48 * 128 // 4
+    assert 1.3e9 * 2 / 8 / 1e6 == pytest.approx(325.0)
+    assert 2 / 16 == 1 / 8
+
+
+# ---------------------------------------------------------------------------
+# Widely-linear transform
+# ---------------------------------------------------------------------------
+def test_widely_linear_hand_example():
+    g = {r[0]: r[1:] for r in read_golden("widely_linear_2x2.txt")}
+    R = np.array([float(v) for v in g["R"]]).reshape(2, 2)
+    U, W = O.widely_linear_from_real(R)
+    assert U[0, 0] == complex(*[float(v) for v in g["U"]])
+    assert W[0, 0] == complex(*[float(v) for v in g["W"]])
+
+
+def test_widely_linear_identity_fp64():
+    """R [x_re; x_im] = U x + W conj(x), to 1e-12 relative, on random shapes."""
+    rng = np.random.default_rng(12)
+    for (n, m) in ((3, 5), (16, 8), (40, 64)):
+        R = rng.standard_normal((2 * n, 2 * m))
+        U, W = O.widely_linear_from_real(R)
+        xr, xi = rng.standard_normal(m), rng.standard_normal(m)
+        y_real = R @ np.concatenate([xr, xi])
+        x = xr + 1j * xi
+        y = U @ x + W @ np.conj(x)
+        scale = np.abs(R) @ np.concatenate([np.abs(xr), np.abs(xi)])
+        assert np.max(np.abs(y.real - y_real[:n]) / scale[:n]) <= 1e-12
+        assert np.max(np.abs(y.imag - y_real[n:]) / scale[n:]) <= 1e-12
+
+
+def test_widely_linear_fp32_planes_are_exactly_rounded():
+    """Each fp32 plane entry is the exact rational (R_ab +- R_cd)/2 rounded to nearest-even."""
+    rng = np.random.default_rng(13)
+    R = (0.02 * rng.standard_normal((6, 8))).astype(np.float32)
+    ur, ui, wr, wi = O.widely_linear_planes_fp32(R)
+    n, m = 3, 4
+    for i in range(n):
+        for j in range(m):
+            r11, r12 = Fraction(float(R[i, j])), Fraction(float(R[i, j + m]))
+            r21, r22 = Fraction(float(R[i + n, j])), Fraction(float(R[i + n, j + m]))
+            for got, exact in ((ur, (r11 + r22) / 2), (ui, (r21 - r12) / 2),
+                               (wr, (r11 - r22) / 2), (wi, (r12 + r21) / 2)):
+                # nearest fp32 to the exact rational: compare with both neighbours
+                g = Fraction(float(got[i, j]))
+                up = Fraction(float(np.nextafter(got[i, j], np.float32(np.inf))))
+                dn = Fraction(float(np.nextafter(got[i, j], np.float32(-np.inf))))
+                assert abs(g - exact) <= abs(up - exact) and abs(g - exact) <= abs(dn - exact)
+
+
+def test_widely_linear_rounded_planes_meet_page_bound():
+    """With fp32-rounded U, W the identity still holds far inside the 1e-6 conversion bound
+    ("Fairy2i write-up" §5.2)."""
+    rng = np.random.default_rng(14)
+    R = (0.02 * rng.standard_normal((64, 96))).astype(np.float32)
+    ur, ui, wr, wi = (p.astype(np.float64) for p in O.widely_linear_planes_fp32(R))
+    xr, xi = rng.standard_normal(48), rng.standard_normal(48)
+    x = xr + 1j * xi
+    y = (ur + 1j * ui) @ x + (wr + 1j * wi) @ np.conj(x)
+    y_real = R.astype(np.float64) @ np.concatenate([xr, xi])
+    rel = np.max(np.abs(np.concatenate([y.real, y.imag]) - y_real)) / np.max(np.abs(y_real))
+    assert rel < 1e-6
+
+
+# ---------------------------------------------------------------------------
+# Product
+# ---------------------------------------------------------------------------
+def test_product_hand_example():
+    g = {r[0]: r[1:] for r in read_golden("product_example.txt")}
+    cu = O.pack_codes(np.array([[int(v) for v in g["u_codes"]]], np.uint8))[None]
+    cw = O.pack_codes(np.array([[int(v) for v in g["w_codes"]]], np.uint8))[None]
+    su = np.array([[float(v) for v in g["u_scales"]]], np.float32)
+    sw = np.array([[float(v) for v in g["w_scales"]]], np.float32)
+    xr = np.array([[float(v) for v in g["x_re"]]])
+    xi = np.array([[float(v) for v in g["x_im"]]])
+    yu = O.product(cu, su, None, None, xr, xi)
+    y = O.product(cu, su, cw, sw, xr, xi)
+    assert yu[0, 0] == complex(*[float(v) for v in g["y_u"]])
+    assert y[0, 0] == complex(*[float(v) for v in g["y"]])
+
+
+def test_product_brute_force_all_code_rows():
+    """K = 4: all 256 code rows, against direct multiplication by codebook values as Python complex."""
+    rng = np.random.default_rng(15)
+    rows = np.array([[(r >> (2 * q)) & 3 for q in range(4)] for r in range(256)], np.uint8)
+    T = 2
+    codes = [rows, rows[::-1].copy()]
+    scales = np.array([[0.7, 1.3], [0.11, 0.05]], np.float32)
+    wcodes = [rows[rng.permutation(256)], rows[rng.permutation(256)]]
+    wscales = np.array([[0.3, 0.9], [0.02, 0.08]], np.float32)
+    xr = O.bf16_round(rng.standard_normal((3, 4)).astype(np.float32))
+    xi = O.bf16_round(rng.standard_normal((3, 4)).astype(np.float32))
+    y = O.product(np.stack([O.pack_codes(c) for c in codes]), scales,
+                  np.stack([O.pack_codes(c) for c in wcodes]), wscales, xr, xi)
+    for bb in range(3):
+        x = [complex(float(xr[bb, j]), float(xi[bb, j])) for j in range(4)]
+        for n in range(256):
+            acc = 0j
+            for t in range(T):
+                for j in range(4):
+                    cu = O.CODEBOOK[codes[t][n, j]]
+                    cw = O.CODEBOOK[wcodes[t][n, j]]
+                    wu = complex(float(scales[t, 0]) * cu.real, float(scales[t, 1]) * cu.imag)
+                    ww = complex(float(wscales[t, 0]) * cw.real, float(wscales[t, 1]) * cw.imag)
+                    acc += wu * x[j] + ww * x[j].conjugate()
+            assert abs(y[bb, n] - acc) <= 1e-12 * (1 + abs(acc))
+
+
+def test_product_one_hot_and_all_ones():
+    rng = np.random.default_rng(16)
+    k = rng.integers(0, 4, size=(8, 12), dtype=np.uint8)
+    packed = O.pack_codes(k)[None]
+    sc = np.array([[0.5, 0.25]], np.float32)
+    W_hat = O.dequantize(packed, sc)
+    for j in range(12):
+        xr = np.zeros((1, 12))
+        xr[0, j] = 1.0
+        y = O.product(packed, sc, None, None, xr, np.zeros((1, 12)))
+        np.testing.assert_array_equal(y[0], W_hat[:, j])
+    ones = O.pack_codes(np.zeros((3, 12), np.uint8))[None]
+    xr = O.bf16_round(rng.standard_normal((1, 12)).astype(np.float32))
+    xi = O.bf16_round(rng.standard_normal((1, 12)).astype(np.float32))
+    y = O.product(ones, sc, None, None, xr, xi)
+    want = 0.5 * (np.sum(xr.astype(np.float64)) + 1j * np.sum(xi.astype(np.float64)))
+    assert np.allclose(y[0], want, rtol=1e-14, atol=0)
+
+
+def test_product_rows_subset_matches_full():
+    rng = np.random.default_rng(17)
+    k = rng.integers(0, 4, size=(2, 20, 16), dtype=np.uint8)
+    packed = np.stack([O.pack_codes(k[0]), O.pack_codes(k[1])])
+    sc = np.array([[0.5, 0.25], [0.1, 0.2]], np.float32)
+    xr = rng.standard_normal((2, 16))
+    xi = rng.standard_normal((2, 16))
+    full = O.product(packed, sc, packed, sc[::-1], xr, xi)
+    rows = np.array([3, 0, 19])
+    sub = O.product_rows(packed, sc, packed, sc[::-1], xr, xi, rows)
+    np.testing.assert_allclose(sub, full[:, rows], rtol=1e-14)
+
+
+def test_tolerance_bound_formula():
+    su = np.array([[1.0, 2.0]], np.float32)
+    sw = np.array([[0.5, 0.5]], np.float32)
+    xr = np.array([[1.0, -2.0]])
+    xi = np.array([[0.0, 3.0]])
+    assert O.tolerance_bound(su, sw, xr, xi)[0] == pytest.approx(1e-5 * 4.0 * 6.0)
+    assert O.tolerance_bound(su, None, xr, xi)[0] == pytest.approx(1e-5 * 3.0 * 6.0)
