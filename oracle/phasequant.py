@@ -76,14 +76,10 @@ def phase_code(a, b):
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)
     aa, ab = np.abs(a), np.abs(b)
-    k = np.zeros(np.broadcast(a, b).shape, dtype=np.uint8)
     k1 = (b > aa) | ((a == b) & (b > 0))
     k2 = (-a > ab) | ((b == -a) & (a < 0))
     k3 = (-b > aa) | ((a == b) & (b < 0))
-    k[k1] = 1
-    k[k2] = 2
-    k[k3] = 3
-    return k
+    return np.where(k1, np.uint8(1), np.where(k2, np.uint8(2), np.where(k3, np.uint8(3), np.uint8(0))))
 
 
 def code_to_br_bi(k):

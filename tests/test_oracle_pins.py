@@ -414,3 +414,45 @@ def test_tolerance_bound_formula():
     xi = np.array([[0.0, 3.0]])
     assert O.tolerance_bound(su, sw, xr, xi)[0] == pytest.approx(1e-5 * 4.0 * 6.0)
     assert O.tolerance_bound(su, None, xr, xi)[0] == pytest.approx(1e-5 * 3.0 * 6.0)
+
+
+# ---------------------------------------------------------------------------
+# The plain-C restatement of a stage (used for full-size runs) against the above
+# ---------------------------------------------------------------------------
+def test_c_stage_matches_hand_example():
+    from oracle import cref
+    g = {r[0]: r[1:] for r in read_golden("two_stage_example.txt")}
+    w_re = np.array([float(v) for v in g["w_re"]], np.float32)[None, :]
+    w_im = np.array([float(v) for v in g["w_im"]], np.float32)[None, :]
+    codes, scales = cref.quantize_tensor(w_re, w_im, 2)
+    assert list(codes[0, 0]) == [int(v, 16) for v in g["bytes1"]]
+    assert list(codes[1, 0]) == [int(v, 16) for v in g["bytes2"]]
+    assert scales[1, 0] == np.float32(Fraction(17, 12)) and scales[1, 1] == np.float32(1.7)
+
+
+def test_c_stage_matches_numpy_oracle():
+    from oracle import cref
+    rng = np.random.default_rng(21)
+    for (N, K, T) in ((7, 12, 1), (33, 64, 3), (64, 256, 4)):
+        wr = (0.02 * rng.standard_normal((N, K))).astype(np.float32)
+        wi = (0.03 * rng.standard_normal((N, K))).astype(np.float32)
+        wr[0, :3] = [np.nan, np.inf, 0.0]
+        wi[1, :2] = [1e-3, 1e-3]
+        wr[1, :2] = [1e-3, -1e-3]
+        c1, s1 = cref.quantize_tensor(wr, wi, T)
+        c2, s2, _ = O.quantize_tensor(wr, wi, T)
+        np.testing.assert_array_equal(c1, c2)
+        np.testing.assert_allclose(s1, s2, rtol=1e-7, atol=0)
+
+
+def test_c_near_boundary_flags_match_numpy():
+    from oracle import cref
+    rng = np.random.default_rng(22)
+    wr = (0.02 * rng.standard_normal((16, 64))).astype(np.float32)
+    wi = wr.copy()
+    wi[:, ::2] = (0.02 * rng.standard_normal((16, 32))).astype(np.float32)
+    codes, scales = cref.quantize_tensor(wr, wi, 2)
+    _, _, near = cref.stage(wr, wi, 1, codes[:1].reshape(1, -1), scales[:1], want_near=True)
+    a, b = O.residual_after(wr, wi, [O.unpack_codes(codes[0])], [tuple(scales[0])])
+    want = O.near_boundary_mask(a, b, float(np.sum(scales[0].astype(np.float64))))
+    np.testing.assert_array_equal(near.reshape(16, 64).astype(bool), want)
