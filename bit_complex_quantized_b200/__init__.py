@@ -1,0 +1,23 @@
+"""B200-native PhaseQuant and multiplication-free complex GEMV/GEMM (libifq).
+
+The compute path is the CUDA library libifq.so (include/ifq.h); this package
+holds its ctypes binding (_lib), the in-tree build script (build) and the
+seeded synthetic workload generator (workloads).
+"""
+from ._lib import (  # noqa: F401
+    EXPORTED,
+    IFQ_DEV_NONFINITE,
+    IFQ_DEV_TIMEOUT,
+    IFQ_MAX_GEMV_BATCH,
+    IFQ_MAX_GROUP,
+    IFQ_MAX_STAGES,
+    IfqError,
+    LIB_PATH,
+    ifq_gemm,
+    ifq_gemv,
+    ifq_quantize_pack,
+    ifq_quantize_workspace_bytes,
+    ifq_status_string,
+    ifq_widely_linear_from_real,
+    load,
+)

@@ -1,0 +1,155 @@
+"""ctypes binding of libifq (include/ifq.h): argument marshalling only.
+
+Each function takes torch tensors that already live on the GPU, passes their
+device pointers and sizes to the C ABI function of the same name, and raises
+IfqError on a non-OK status.  No arithmetic of the method happens here, and
+there is no fallback: if libifq.so is missing, loading fails loudly.
+"""
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libifq.so")
+
+IFQ_MAX_STAGES = 8
+IFQ_MAX_GEMV_BATCH = 16
+IFQ_MAX_GROUP = 32
+IFQ_DEV_NONFINITE = 0x1
+IFQ_DEV_TIMEOUT = 0x2
+
+EXPORTED = (
+    "ifq_status_string",
+    "ifq_widely_linear_from_real",
+    "ifq_quantize_workspace_bytes",
+    "ifq_quantize_pack",
+    "ifq_gemv",
+    "ifq_gemm",
+)
+
+STATUS_NAMES = {
+    0: "IFQ_OK", 1: "IFQ_ERR_NULL", 2: "IFQ_ERR_SHAPE", 3: "IFQ_ERR_ALIGN", 4: "IFQ_ERR_STAGES",
+    5: "IFQ_ERR_BATCH", 6: "IFQ_ERR_WORKSPACE", 7: "IFQ_ERR_CUDA", 8: "IFQ_ERR_UNSUPPORTED", 9: "IFQ_ERR_COUNT",
+}
+
+
+class IfqError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+class QTensor(ctypes.Structure):
+    _fields_ = [("w_re", ctypes.c_void_p), ("w_im", ctypes.c_void_p), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int64), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+class Layer(ctypes.Structure):
+    _fields_ = [("codes_u", ctypes.c_void_p), ("scales_u", ctypes.c_void_p), ("codes_w", ctypes.c_void_p),
+                ("scales_w", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("x_re", ctypes.c_void_p), ("x_im", ctypes.c_void_p), ("y_re", ctypes.c_void_p),
+                ("y_im", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load():
+    """Load libifq.so (built in-tree); raises if it is absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with python -m bit_complex_quantized_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    i64, i32, vp, sz = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+    lib.ifq_status_string.restype = ctypes.c_char_p
+    lib.ifq_status_string.argtypes = [i32]
+    lib.ifq_widely_linear_from_real.restype = i32
+    lib.ifq_widely_linear_from_real.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp]
+    lib.ifq_quantize_workspace_bytes.restype = sz
+    lib.ifq_quantize_workspace_bytes.argtypes = [ctypes.POINTER(QTensor), i32, i32]
+    lib.ifq_quantize_pack.restype = i32
+    lib.ifq_quantize_pack.argtypes = [ctypes.POINTER(QTensor), i32, i32, vp, sz, vp, vp]
+    lib.ifq_gemv.restype = i32
+    lib.ifq_gemv.argtypes = [ctypes.POINTER(Layer), i32, i32, i32, vp, vp]
+    lib.ifq_gemm.restype = i32
+    lib.ifq_gemm.argtypes = [ctypes.POINTER(Layer), i32, i32, i64, vp, vp]
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status):
+    if status != 0:
+        raise IfqError(status, load().ifq_status_string(status).decode())
+
+
+def ifq_status_string(status):
+    return load().ifq_status_string(int(status)).decode()
+
+
+def ifq_widely_linear_from_real(R, U_re, U_im, W_re, W_im, stream=None):
+    """R: float32 [2n][2m]; outputs float32 [n][m] (all on the device)."""
+    rows, cols = R.shape
+    _check(load().ifq_widely_linear_from_real(_ptr(R), rows, cols, _ptr(U_re), _ptr(U_im), _ptr(W_re), _ptr(W_im),
+                                              _stream(stream)))
+
+
+def _qtensors(tensors):
+    arr = (QTensor * len(tensors))()
+    for i, t in enumerate(tensors):
+        w_re, w_im, codes, scales = t
+        arr[i] = QTensor(w_re.data_ptr(), w_im.data_ptr(), w_re.shape[0], w_re.shape[1], codes.data_ptr(),
+                         scales.data_ptr())
+    return arr
+
+
+def ifq_quantize_workspace_bytes(tensors, T):
+    """tensors: list of (w_re, w_im, codes, scales)."""
+    return int(load().ifq_quantize_workspace_bytes(_qtensors(tensors), len(tensors), T))
+
+
+def ifq_quantize_pack(tensors, T, workspace, dev_status=None, stream=None, workspace_bytes=None):
+    """tensors: list of (w_re [N][K] f32, w_im, codes u8 [T][N][K/4], scales f32 [T][2])."""
+    arr = _qtensors(tensors)
+    nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check(load().ifq_quantize_pack(arr, len(tensors), T, _ptr(workspace), nbytes, _ptr(dev_status),
+                                    _stream(stream)))
+
+
+def _layers(layers):
+    arr = (Layer * len(layers))()
+    for i, d in enumerate(layers):
+        arr[i] = Layer(d["codes_u"].data_ptr(), d["scales_u"].data_ptr(),
+                       None if d.get("codes_w") is None else d["codes_w"].data_ptr(),
+                       None if d.get("scales_w") is None else d["scales_w"].data_ptr(),
+                       d["N"], d["K"], d["x_re"].data_ptr(), d["x_im"].data_ptr(), d["y_re"].data_ptr(),
+                       d["y_im"].data_ptr())
+    return arr
+
+
+def ifq_gemv(layers, T, B, dev_status=None, stream=None):
+    """layers: list of dicts with codes_u, scales_u, codes_w, scales_w (or None), N, K,
+    x_re, x_im (bf16 [B][K]), y_re, y_im (float32 [B][N])."""
+    _check(load().ifq_gemv(_layers(layers), len(layers), T, B, _ptr(dev_status), _stream(stream)))
+
+
+def ifq_gemm(layers, T, M, dev_status=None, stream=None):
+    """As ifq_gemv with x [M][K] and y [M][N]."""
+    _check(load().ifq_gemm(_layers(layers), len(layers), T, M, _ptr(dev_status), _stream(stream)))
+
+
+# Raw entry point for callers that build ctypes descriptors themselves.
+def raw():
+    return load()

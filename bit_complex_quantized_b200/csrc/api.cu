@@ -1,0 +1,125 @@
+// C ABI of libifq: argument validation, then one enqueue per entry point.
+// Every error is returned before anything is launched.
+#include <cuda_runtime.h>
+
+#include "../../include/ifq.h"
+#include "ifq_internal.h"
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline cudaStream_t as_stream(ifq_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// The kernels use sm_100a instructions (tcgen05, TMA); refuse other devices.
+ifq_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return IFQ_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return IFQ_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return IFQ_ERR_CUDA;
+  if (major != 10 || minor != 0) return IFQ_ERR_UNSUPPORTED;
+  return IFQ_OK;
+}
+
+ifq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? IFQ_OK : IFQ_ERR_CUDA; }
+
+ifq_status check_layers(const ifq_layer* L, int count, int T) {
+  if (!L) return IFQ_ERR_NULL;
+  if (count < 1 || count > IFQ_MAX_GROUP) return IFQ_ERR_COUNT;
+  if (T < 1 || T > IFQ_MAX_STAGES) return IFQ_ERR_STAGES;
+  for (int i = 0; i < count; ++i) {
+    const ifq_layer& l = L[i];
+    if (!l.codes_u || !l.scales_u || !l.x_re || !l.x_im || !l.y_re || !l.y_im) return IFQ_ERR_NULL;
+    if ((l.codes_w == nullptr) != (l.scales_w == nullptr)) return IFQ_ERR_NULL;
+    if (l.N < 1 || l.K < 64 || (l.K % 64) != 0) return IFQ_ERR_SHAPE;
+    if (l.N > (int64_t)1 << 30 || l.K > (int64_t)1 << 30) return IFQ_ERR_SHAPE;
+    if (!aligned16(l.codes_u) || (l.codes_w && !aligned16(l.codes_w)) || !aligned16(l.x_re) || !aligned16(l.x_im) ||
+        !aligned16(l.y_re) || !aligned16(l.y_im) || (reinterpret_cast<uintptr_t>(l.scales_u) & 3u) ||
+        (reinterpret_cast<uintptr_t>(l.scales_w) & 3u))
+      return IFQ_ERR_ALIGN;
+  }
+  return IFQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ifq_status_string(ifq_status s) {
+  switch (s) {
+    case IFQ_OK: return "ok";
+    case IFQ_ERR_NULL: return "a required pointer is NULL";
+    case IFQ_ERR_SHAPE: return "invalid shape";
+    case IFQ_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case IFQ_ERR_STAGES: return "stage count T outside 1..8";
+    case IFQ_ERR_BATCH: return "batch outside the supported range";
+    case IFQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case IFQ_ERR_CUDA: return "CUDA runtime error";
+    case IFQ_ERR_UNSUPPORTED: return "device is not sm_100";
+    case IFQ_ERR_COUNT: return "descriptor count outside 1..32";
+  }
+  return "unknown status";
+}
+
+ifq_status ifq_widely_linear_from_real(const float* R, int64_t rows, int64_t cols, float* U_re, float* U_im,
+                                       float* W_re, float* W_im, ifq_stream_t stream) {
+  if (!R || !U_re || !U_im || !W_re || !W_im) return IFQ_ERR_NULL;
+  if (rows < 2 || cols < 2 || (rows & 1) || (cols & 1)) return IFQ_ERR_SHAPE;
+  if (!aligned16(R) || !aligned16(U_re) || !aligned16(U_im) || !aligned16(W_re) || !aligned16(W_im))
+    return IFQ_ERR_ALIGN;
+  ifq_status st = check_device();
+  if (st != IFQ_OK) return st;
+  return from_cuda(ifq::launch_widely_linear(R, rows / 2, cols / 2, U_re, U_im, W_re, W_im, as_stream(stream)));
+}
+
+size_t ifq_quantize_workspace_bytes(const ifq_qtensor* tensors, int count, int T) {
+  (void)T;
+  if (!tensors || count < 1 || count > IFQ_MAX_GROUP) return 0;
+  for (int i = 0; i < count; ++i)
+    if (tensors[i].N < 1 || tensors[i].K < 4 || tensors[i].K % 4) return 0;
+  return ifq::quant_workspace_bytes(tensors, count);
+}
+
+ifq_status ifq_quantize_pack(const ifq_qtensor* tensors, int count, int T, void* workspace, size_t workspace_bytes,
+                             uint32_t* dev_status, ifq_stream_t stream) {
+  if (!tensors) return IFQ_ERR_NULL;
+  if (count < 1 || count > IFQ_MAX_GROUP) return IFQ_ERR_COUNT;
+  if (T < 1 || T > IFQ_MAX_STAGES) return IFQ_ERR_STAGES;
+  for (int i = 0; i < count; ++i) {
+    const ifq_qtensor& t = tensors[i];
+    if (!t.w_re || !t.w_im || !t.codes || !t.scales) return IFQ_ERR_NULL;
+    if (t.N < 1 || t.K < 4 || (t.K % 4) != 0) return IFQ_ERR_SHAPE;
+    if (t.K > (int64_t)1 << 30 || t.N > ((int64_t)1 << 40) / t.K) return IFQ_ERR_SHAPE;
+    if (!aligned16(t.w_re) || !aligned16(t.w_im) || !aligned16(t.codes) || (reinterpret_cast<uintptr_t>(t.scales) & 3u))
+      return IFQ_ERR_ALIGN;
+  }
+  if (!workspace || workspace_bytes < ifq::quant_workspace_bytes(tensors, count)) return IFQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return IFQ_ERR_ALIGN;
+  ifq_status st = check_device();
+  if (st != IFQ_OK) return st;
+  return from_cuda(ifq::launch_quantize(tensors, count, T, workspace, dev_status, as_stream(stream)));
+}
+
+ifq_status ifq_gemv(const ifq_layer* layers, int count, int T, int B, uint32_t* dev_status, ifq_stream_t stream) {
+  ifq_status st = check_layers(layers, count, T);
+  if (st != IFQ_OK) return st;
+  if (B < 1 || B > IFQ_MAX_GEMV_BATCH) return IFQ_ERR_BATCH;
+  st = check_device();
+  if (st != IFQ_OK) return st;
+  return from_cuda(ifq::launch_gemv(layers, count, T, B, dev_status, as_stream(stream)));
+}
+
+ifq_status ifq_gemm(const ifq_layer* layers, int count, int T, int64_t M, uint32_t* dev_status,
+                    ifq_stream_t stream) {
+  ifq_status st = check_layers(layers, count, T);
+  if (st != IFQ_OK) return st;
+  if (M < 1 || M > ((int64_t)1 << 31) - 128) return IFQ_ERR_BATCH;
+  for (int i = 0; i < count; ++i)
+    if ((int64_t)T * layers[i].N > ((int64_t)1 << 31) - 64) return IFQ_ERR_SHAPE;
+  st = check_device();
+  if (st != IFQ_OK) return st;
+  return from_cuda(ifq::launch_gemm(layers, count, T, M, dev_status, as_stream(stream)));
+}
+
+}  // extern "C"

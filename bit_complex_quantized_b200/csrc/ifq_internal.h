@@ -1,0 +1,24 @@
+// Internal launch interfaces between the C-ABI layer (api.cu) and the kernel
+// files.  Arguments are validated by the caller; these only enqueue work.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/ifq.h"
+
+namespace ifq {
+
+cudaError_t launch_widely_linear(const float* R, int64_t n, int64_t m, float* U_re, float* U_im, float* W_re,
+                                 float* W_im, cudaStream_t s);
+
+// Quantizer: per-tensor block counts and workspace layout.
+int64_t quant_blocks_for(int64_t N, int64_t K);
+size_t quant_workspace_bytes(const ifq_qtensor* t, int count);
+cudaError_t launch_quantize(const ifq_qtensor* t, int count, int T, void* ws, uint32_t* dev_status, cudaStream_t s);
+
+cudaError_t launch_gemv(const ifq_layer* L, int count, int T, int B, uint32_t* dev_status, cudaStream_t s);
+
+cudaError_t launch_gemm(const ifq_layer* L, int count, int T, int64_t M, uint32_t* dev_status, cudaStream_t s);
+
+}  // namespace ifq

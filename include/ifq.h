@@ -1,0 +1,179 @@
+/*
+ * ifq.h -- C ABI of libifq: PhaseQuant quantization of complex weights to the
+ * fourth roots of unity {1, i, -1, -i} and the multiplication-free complex
+ * product that consumes the codes, on one NVIDIA B200 (sm_100a).
+ *
+ * Method sources, by page and section:
+ *   "Fairy2i write-up" (hotelren.com): §2.1 widely-linear transform y = Ux + W conj(x),
+ *     §3.1 phase rule, §3.2 axis-aligned scales, §4.1 recursive residual stages,
+ *     §4.2 multiplication-free product.
+ *   "iFairy article" (bestcxt.com): §二.1 codebook and 2-bit storage, §二.2 GEMM by add/sub/swap.
+ *   "iFairy talk notes" (43b.com.cn): §2.2.2 phase rule, §2.3.1 x i = swap + negate.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers into caller-owned memory.  The
+ *     library allocates nothing, keeps no state between calls, never
+ *     synchronizes the host, and enqueues all work on the caller's stream.
+ *     Descriptor arrays (ifq_qtensor*, ifq_layer*) are HOST pointers; they
+ *     are read during the call and may be freed when it returns.
+ *   - Every argument error is reported by the return value before anything
+ *     is enqueued.  Conditions that only the GPU can see set bits in the
+ *     caller's device status word (dev_status), which the caller reads after
+ *     synchronizing; no kernel traps or asserts.
+ *   - Complex tensors are planar: a real plane and an imaginary plane.
+ *   - Code k in {0,1,2,3} stands for the codebook entry [1, i, -1, -i][k]
+ *     (the list order of the §3.1 phase-rule sketch).  Bit 0 of k is the axis
+ *     (0: real, +-1; 1: imaginary, +-i), bit 1 the sign.
+ *   - Packed codes: uint8 [T][N][K/4], row-major; code j of row n of stage t
+ *     is bits 2(j%4) and 2(j%4)+1 of byte [t][n][j/4].  2 bits per complex
+ *     weight per stage.
+ *   - Scales: float32 [T][2] = {s_re, s_im} per stage, per tensor (§3.2).
+ *     Stage t's dequantized weight is w_hat_t = s_re Re(b) + i s_im Im(b).
+ *   - Activations: bf16 bit patterns, planar, token-major [B or M][K].
+ *     Outputs: float32, planar, token-major [B or M][N], OVERWRITTEN.
+ */
+#ifndef IFQ_H
+#define IFQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t passed as an opaque pointer (NULL = the legacy default stream). */
+typedef void* ifq_stream_t;
+
+typedef enum {
+  IFQ_OK = 0,
+  IFQ_ERR_NULL = 1,        /* a required pointer is NULL */
+  IFQ_ERR_SHAPE = 2,       /* a size is zero, negative, odd where it must be even, or not a multiple the call needs */
+  IFQ_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
+  IFQ_ERR_STAGES = 4,      /* T outside 1..IFQ_MAX_STAGES */
+  IFQ_ERR_BATCH = 5,       /* B outside 1..IFQ_MAX_GEMV_BATCH, or M < 1 */
+  IFQ_ERR_WORKSPACE = 6,   /* workspace NULL or smaller than ifq_quantize_workspace_bytes() */
+  IFQ_ERR_CUDA = 7,        /* a CUDA runtime call failed (launch error, no device, ...) */
+  IFQ_ERR_UNSUPPORTED = 8, /* the device is not sm_100 */
+  IFQ_ERR_COUNT = 9        /* descriptor count outside 1..IFQ_MAX_GROUP */
+} ifq_status;
+
+#define IFQ_MAX_STAGES 8
+#define IFQ_MAX_GEMV_BATCH 16
+#define IFQ_MAX_GROUP 32
+
+/* Device status bits, OR-ed into *dev_status by kernels. */
+#define IFQ_DEV_NONFINITE 0x1u /* a weight was NaN or Inf; it was quantized as 0 (code 0) */
+#define IFQ_DEV_TIMEOUT 0x2u   /* a bounded pipeline wait gave up; outputs of that call are invalid */
+
+const char* ifq_status_string(ifq_status s);
+
+/* ---------------------------------------------------------------------------
+ * ifq_widely_linear_from_real  ("Fairy2i write-up" §2.1)
+ *
+ * Splits a real layer R (rows = 2n outputs, cols = 2m inputs, float32
+ * row-major) into complex n x m matrices U and W with R [x_re; x_im] =
+ * U x + W conj(x):
+ *   U_re = (R11 + R22)/2, U_im = (R21 - R12)/2,
+ *   W_re = (R11 - R22)/2, W_im = (R12 + R21)/2,
+ * with R11 = R[:n,:m], R12 = R[:n,m:], R21 = R[n:,:m], R22 = R[n:,m:].
+ * Each output is the float32 sum or difference rounded to nearest-even, then
+ * halved, which equals the exact value rounded once.
+ *
+ *   R                     [rows][cols] float32, device, read-only
+ *   rows, cols            even, >= 2
+ *   U_re, U_im, W_re, W_im  [rows/2][cols/2] float32, device, written
+ * Pointers must be 16-byte aligned.  The four outputs must not overlap R.
+ * ------------------------------------------------------------------------- */
+ifq_status ifq_widely_linear_from_real(const float* R, int64_t rows, int64_t cols,
+                                       float* U_re, float* U_im, float* W_re, float* W_im,
+                                       ifq_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * ifq_quantize_pack  ("Fairy2i write-up" §3.1, §3.2, §4.1)
+ *
+ * T-stage PhaseQuant of `count` complex tensors.  Stage t quantizes the
+ * residual r_t = w - sum_{u<t} w_hat_u (r_1 = w), computed in float64 from w
+ * and the codes and float32 scales of the earlier stages:
+ *   k = sector of r_t: floor(2 arg(r)/pi + 0.5) mod 4, evaluated exactly by
+ *       comparisons (a tie on a diagonal goes counter-clockwise; r = 0 -> 0);
+ *   s_re = mean |Re r| over entries coded +-1, s_im = mean |Im r| over
+ *       entries coded +-i (float64 sums, rounded to float32; 0 if none).
+ * An entry with a NaN or Inf part is quantized as 0 and sets IFQ_DEV_NONFINITE.
+ * Sums are reduced in a fixed order, so results are bit-reproducible.
+ *
+ *   tensors[i].w_re, w_im   [N][K] float32, device, read-only, 16-byte aligned
+ *   tensors[i].N, K         N >= 1, K >= 4, K % 4 == 0
+ *   tensors[i].codes        [T][N][K/4] uint8, device, written, 16-byte aligned
+ *   tensors[i].scales       [T][2] float32, device, written
+ *   count                   1..IFQ_MAX_GROUP tensors, processed together
+ *   T                       1..IFQ_MAX_STAGES
+ *   workspace               device scratch of ifq_quantize_workspace_bytes()
+ *                           bytes, 16-byte aligned, owned by the caller; no
+ *                           initial contents needed; must not be used by
+ *                           anything else until the enqueued work finishes
+ *   dev_status              device uint32, bits OR-ed in (may be NULL)
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  const float* w_re;
+  const float* w_im;
+  int64_t N;
+  int64_t K;
+  uint8_t* codes;
+  float* scales;
+} ifq_qtensor;
+
+size_t ifq_quantize_workspace_bytes(const ifq_qtensor* tensors, int count, int T);
+
+ifq_status ifq_quantize_pack(const ifq_qtensor* tensors, int count, int T, void* workspace,
+                             size_t workspace_bytes, uint32_t* dev_status, ifq_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Product layers ("Fairy2i write-up" §2.1, §4.2; "iFairy article" §二.2)
+ *
+ *   y = sum_t ( U_hat_t x + W_hat_t conj(x) ),  per token,
+ * where U_hat_t, W_hat_t are stage t of the two code sets.  Each code adds or
+ * subtracts the real or imaginary part of x into a per-class float32
+ * accumulator (no multiplications by weights); the scales are applied once per
+ * (stage, branch) in the epilogue.
+ *
+ *   codes_u, scales_u   stage codes and scales of U (required)
+ *   codes_w, scales_w   of W, applied to conj(x); both NULL = no conjugate branch
+ *   N, K                outputs, inputs: N >= 1, K >= 64, K % 64 == 0
+ *   x_re, x_im          [rows][K] bf16 bit patterns, device, 16-byte aligned
+ *   y_re, y_im          [rows][N] float32, device, overwritten
+ * rows = B for ifq_gemv and M for ifq_gemm.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  const uint8_t* codes_u;
+  const float* scales_u;
+  const uint8_t* codes_w;
+  const float* scales_w;
+  int64_t N;
+  int64_t K;
+  const uint16_t* x_re;
+  const uint16_t* x_im;
+  float* y_re;
+  float* y_im;
+} ifq_layer;
+
+/* Decode product for B = 1..IFQ_MAX_GEMV_BATCH tokens per layer; all `count`
+ * layers (1..IFQ_MAX_GROUP) run in one launch.  Codes stream from HBM once;
+ * the per-code work is a sign flip and an axis select feeding float32
+ * accumulation.  dev_status may be NULL. */
+ifq_status ifq_gemv(const ifq_layer* layers, int count, int T, int B, uint32_t* dev_status,
+                    ifq_stream_t stream);
+
+/* Prefill product for M >= 1 tokens (meant for M >= 128) on the tensor cores:
+ * codes are expanded in shared memory to exact {-2, 0, +2} bf16 operands, the
+ * +-1 and +-i classes accumulate in separate float32 TMEM accumulators, and the
+ * scales are applied per (stage, branch) in the epilogue.  Layers run one after
+ * another on the stream.  dev_status may be NULL (timeouts then go unreported). */
+ifq_status ifq_gemm(const ifq_layer* layers, int count, int T, int64_t M, uint32_t* dev_status,
+                    ifq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* IFQ_H */

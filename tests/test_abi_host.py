@@ -1,0 +1,114 @@
+"""Host-side checks of libifq (no GPU needed): the shared library loads and
+exports every function include/ifq.h declares, and argument errors come back
+as status codes before any CUDA call is made."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bit_complex_quantized_b200 as Q
+from bit_complex_quantized_b200 import _lib as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "ifq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(ifq_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_library_exports_every_declared_function():
+    lib = Q.load()
+    names = _declared_functions()
+    assert len(names) >= 6
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(L.EXPORTED)
+
+
+def test_status_strings():
+    lib = Q.load()
+    for s in range(10):
+        assert lib.ifq_status_string(s)
+    assert Q.ifq_status_string(0) == "ok"
+
+
+FAKE = 0x10000  # non-null, 16-byte aligned, never dereferenced by validation
+
+
+def _layer(**kw):
+    d = dict(codes_u=FAKE, scales_u=FAKE, codes_w=None, scales_w=None, N=64, K=128,
+             x_re=FAKE, x_im=FAKE, y_re=FAKE, y_im=FAKE)
+    d.update(kw)
+    return L.Layer(d["codes_u"], d["scales_u"], d["codes_w"], d["scales_w"], d["N"], d["K"], d["x_re"],
+                   d["x_im"], d["y_re"], d["y_im"])
+
+
+def _call_gemv(layers, T=1, B=1):
+    arr = (L.Layer * max(1, len(layers)))(*layers)
+    return Q.load().ifq_gemv(arr if layers else None, len(layers), T, B, None, None)
+
+
+def _call_gemm(layers, T=1, M=128):
+    arr = (L.Layer * max(1, len(layers)))(*layers)
+    return Q.load().ifq_gemm(arr if layers else None, len(layers), T, M, None, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(codes_u=None), 1), (dict(x_re=None), 1), (dict(y_im=None), 1),
+    (dict(codes_w=FAKE), 1),                       # W codes without W scales
+    (dict(K=100), 2), (dict(K=0), 2), (dict(N=0), 2), (dict(K=32), 2),
+    (dict(codes_u=FAKE + 4), 3), (dict(x_im=FAKE + 2), 3), (dict(scales_u=FAKE + 1), 3),
+])
+def test_gemv_gemm_argument_errors(kw, status):
+    assert _call_gemv([_layer(**kw)]) == status
+    assert _call_gemm([_layer(**kw)]) == status
+
+
+def test_batch_stage_and_count_errors():
+    good = _layer()
+    assert _call_gemv([good], T=0) == 4
+    assert _call_gemv([good], T=9) == 4
+    assert _call_gemv([good], B=0) == 5
+    assert _call_gemv([good], B=17) == 5
+    assert _call_gemm([good], M=0) == 5
+    assert _call_gemv([]) == 1
+    many = [good] * 33
+    arr = (L.Layer * 33)(*many)
+    assert Q.load().ifq_gemv(arr, 33, 1, 1, None, None) == 9
+
+
+def test_quantize_argument_errors():
+    lib = Q.load()
+    qt = L.QTensor(FAKE, FAKE, 64, 128, FAKE, FAKE)
+    arr = (L.QTensor * 1)(qt)
+    need = lib.ifq_quantize_workspace_bytes(arr, 1, 2)
+    assert need > 0
+    assert lib.ifq_quantize_pack(arr, 1, 2, None, need, None, None) == 6
+    assert lib.ifq_quantize_pack(arr, 1, 2, FAKE, need - 1, None, None) == 6
+    assert lib.ifq_quantize_pack(arr, 1, 9, FAKE, need, None, None) == 4
+    assert lib.ifq_quantize_pack(arr, 0, 2, FAKE, need, None, None) == 9
+    bad = (L.QTensor * 1)(L.QTensor(FAKE, FAKE, 64, 126, FAKE, FAKE))
+    assert lib.ifq_quantize_pack(bad, 1, 2, FAKE, need, None, None) == 2
+    assert lib.ifq_quantize_workspace_bytes(bad, 1, 2) == 0
+    mis = (L.QTensor * 1)(L.QTensor(FAKE + 8, FAKE, 64, 128, FAKE, FAKE))
+    assert lib.ifq_quantize_pack(mis, 1, 2, FAKE, need, None, None) == 3
+    nul = (L.QTensor * 1)(L.QTensor(FAKE, None, 64, 128, FAKE, FAKE))
+    assert lib.ifq_quantize_pack(nul, 1, 2, FAKE, need, None, None) == 1
+
+
+def test_workspace_grows_with_tensor_size():
+    lib = Q.load()
+    small = (L.QTensor * 1)(L.QTensor(FAKE, FAKE, 64, 128, FAKE, FAKE))
+    big = (L.QTensor * 2)(L.QTensor(FAKE, FAKE, 4096, 4096, FAKE, FAKE), L.QTensor(FAKE, FAKE, 64, 128, FAKE, FAKE))
+    assert lib.ifq_quantize_workspace_bytes(big, 2, 3) > lib.ifq_quantize_workspace_bytes(small, 1, 3)
+
+
+def test_convert_argument_errors():
+    lib = Q.load()
+    assert lib.ifq_widely_linear_from_real(None, 4, 4, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert lib.ifq_widely_linear_from_real(FAKE, 3, 4, FAKE, FAKE, FAKE, FAKE, None) == 2
+    assert lib.ifq_widely_linear_from_real(FAKE, 4, 0, FAKE, FAKE, FAKE, FAKE, None) == 2
+    assert lib.ifq_widely_linear_from_real(FAKE, 4, 4, FAKE + 4, FAKE, FAKE, FAKE, None) == 3

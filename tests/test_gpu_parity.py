@@ -1,0 +1,318 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle, on the
+five synthetic configurations at full size (sampled outputs where the oracle
+would be slow) and on edge cases."""
+import numpy as np
+import pytest
+import torch
+
+import bit_complex_quantized_b200 as Q
+from bit_complex_quantized_b200 import workloads as W
+import oracle as O
+from ifq_testlib import (DEV, check_convert, check_product, check_quantized, gpu_convert, gpu_quantize,
+                         layer_desc, sample_rows, status_word, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    Q.load()
+
+
+def _complex_cfg_weights(cfg):
+    ws_np = [W.complex_weights(cfg, i) for i in range(len(cfg.layers))]
+    ws_dev = [(to_dev(a), to_dev(b)) for a, b in ws_np]
+    return ws_np, ws_dev
+
+
+def _x(cfg, i, rows):
+    xr, xi = W.activations(cfg, i, rows)
+    return xr.to(DEV), xi.to(DEV), W.bf16_to_f32_numpy(xr), W.bf16_to_f32_numpy(xi)
+
+
+# ---------------------------------------------------------------- config 1
+def test_c1_single_layer_quantize_and_gemv():
+    cfg = W.config("c1")
+    ws_np, ws_dev = _complex_cfg_weights(cfg)
+    st = status_word()
+    (codes, scales), = gpu_quantize(ws_dev, cfg.T, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    cn, sn = codes.cpu().numpy(), scales.cpu().numpy()
+    check_quantized(*ws_np[0], cn, sn, cfg.T)
+    N, K = cfg.layers[0].N, cfg.layers[0].K
+    xr, xi, xrn, xin = _x(cfg, 0, 1)
+    d = layer_desc(codes, scales, None, None, xr, xi, N, K, 1)
+    Q.ifq_gemv([d], cfg.T, 1)
+    torch.cuda.synchronize()
+    check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cn, sn, None, None, xrn, xin)
+
+
+# ---------------------------------------------------------------- config 2
+def test_c2_block_quantize_gemv_b1_b8_and_gemm():
+    cfg = W.config("c2")
+    ws_np, ws_dev = _complex_cfg_weights(cfg)
+    outs = gpu_quantize(ws_dev, cfg.T)
+    torch.cuda.synchronize()
+    host = [(c.cpu().numpy(), s.cpu().numpy()) for c, s in outs]
+    for (wr, wi), (cn, sn) in zip(ws_np, host):
+        check_quantized(wr, wi, cn, sn, cfg.T)
+    for B in (1, 8):
+        descs, xs = [], []
+        for i, spec in enumerate(cfg.layers):
+            xr, xi, xrn, xin = _x(cfg, i, B)
+            xs.append((xrn, xin))
+            descs.append(layer_desc(outs[i][0], outs[i][1], None, None, xr, xi, spec.N, spec.K, B))
+        Q.ifq_gemv(descs, cfg.T, B)
+        torch.cuda.synchronize()
+        for d, (cn, sn), (xrn, xin) in zip(descs, host, xs):
+            check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cn, sn, None, None, xrn, xin)
+    # tensor-core GEMM on the same matrices, M = 200 (one full and one ragged token tile)
+    M = 200
+    descs, xs = [], []
+    for i, spec in enumerate(cfg.layers):
+        xr, xi, xrn, xin = _x(cfg, i, M)
+        xs.append((xrn, xin))
+        descs.append(layer_desc(outs[i][0], outs[i][1], None, None, xr, xi, spec.N, spec.K, M))
+    st = status_word()
+    Q.ifq_gemm(descs, cfg.T, M, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rng = np.random.default_rng(0)
+    for d, (cn, sn), (xrn, xin), spec in zip(descs, host, xs, cfg.layers):
+        rows = sample_rows(spec.N, 96, rng)
+        check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cn, sn, None, None, xrn, xin, rows)
+
+
+# ---------------------------------------------------------------- configs 3 and 4
+@pytest.fixture(scope="module")
+def c3_quantized():
+    """Convert the seven 7B-shaped real layers, quantize all 14 U/W tensors in one
+    grouped call (the config-4 batched quantizer), check conversion and codes."""
+    cfg = W.config("c3")
+    planes, ws_np = [], []
+    for i in range(len(cfg.layers)):
+        R = W.real_weight(cfg, i)
+        p = gpu_convert(R)
+        torch.cuda.synchronize()
+        check_convert(R, p)
+        planes.append(p)
+        del R
+    ws_dev = []
+    for p in planes:
+        ws_dev += [(p[0], p[1]), (p[2], p[3])]
+    st = status_word()
+    outs = gpu_quantize(ws_dev, cfg.T, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    host = [(c.cpu().numpy(), s.cpu().numpy()) for c, s in outs]
+    mism = []
+    for (wr, wi), (cn, sn) in zip(ws_dev, host):
+        mism.append(check_quantized(wr.cpu().numpy(), wi.cpu().numpy(), cn, sn, cfg.T))
+    print("c3 near-boundary mismatches per tensor and stage:", mism)
+    return cfg, outs, host
+
+
+def test_c3_gemv_b1_b16(c3_quantized):
+    cfg, outs, host = c3_quantized
+    rng = np.random.default_rng(3)
+    for B in cfg.batches:
+        descs, xs = [], []
+        for i, spec in enumerate(cfg.layers):
+            xr, xi, xrn, xin = _x(cfg, i, B)
+            xs.append((xrn, xin))
+            (cu, su), (cw, sw) = outs[2 * i], outs[2 * i + 1]
+            descs.append(layer_desc(cu, su, cw, sw, xr, xi, spec.N, spec.K, B))
+        Q.ifq_gemv(descs, cfg.T, B)
+        torch.cuda.synchronize()
+        for i, (d, spec) in enumerate(zip(descs, cfg.layers)):
+            (cun, sun), (cwn, swn) = host[2 * i], host[2 * i + 1]
+            rows = sample_rows(spec.N, 256, rng)
+            check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cun, sun, cwn, swn, *xs[i], rows)
+
+
+def test_c4_gemm_m2048(c3_quantized):
+    cfg3, outs, host = c3_quantized
+    cfg = W.config("c4")
+    M = cfg.prefill_M
+    rng = np.random.default_rng(4)
+    descs, xs = [], []
+    for i, spec in enumerate(cfg.layers):
+        xr, xi, xrn, xin = _x(cfg, i, M)
+        xs.append((xrn, xin))
+        (cu, su), (cw, sw) = outs[2 * i], outs[2 * i + 1]
+        descs.append(layer_desc(cu, su, cw, sw, xr, xi, spec.N, spec.K, M))
+    st = status_word()
+    Q.ifq_gemm(descs, cfg.T, M, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for i, (d, spec) in enumerate(zip(descs, cfg.layers)):
+        (cun, sun), (cwn, swn) = host[2 * i], host[2 * i + 1]
+        rows = sample_rows(spec.N, 48, rng)
+        check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cun, sun, cwn, swn, *xs[i], rows)
+
+
+def test_c3_gemv_and_gemm_agree_on_same_tokens(c3_quantized):
+    cfg, outs, host = c3_quantized
+    i = 6  # down projection, K = 5504
+    spec = cfg.layers[i]
+    B = 16
+    xr, xi, xrn, xin = _x(cfg, i, B)
+    (cu, su), (cw, sw) = outs[2 * i], outs[2 * i + 1]
+    dv = layer_desc(cu, su, cw, sw, xr, xi, spec.N, spec.K, B)
+    dm = layer_desc(cu, su, cw, sw, xr, xi, spec.N, spec.K, B)
+    Q.ifq_gemv([dv], cfg.T, B)
+    Q.ifq_gemm([dm], cfg.T, B)
+    torch.cuda.synchronize()
+    bound = O.tolerance_bound(host[2 * i][1], host[2 * i + 1][1], xrn, xin)[:, None]
+    diff = torch.abs(torch.complex(dv["y_re"].double(), dv["y_im"].double()) -
+                     torch.complex(dm["y_re"].double(), dm["y_im"].double())).cpu().numpy()
+    assert np.all(diff <= 2 * bound)
+
+
+# ---------------------------------------------------------------- config 5
+@pytest.mark.slow
+def test_c5_convert_quantize_gemv():
+    cfg = W.config("c5")
+    rng = np.random.default_rng(5)
+    outs_all, host_all = [], []
+    for i, spec in enumerate(cfg.layers):
+        R = W.real_weight(cfg, i)
+        p = gpu_convert(R)
+        torch.cuda.synchronize()
+        check_convert(R, p, rows=sample_rows(spec.N, 64, rng))
+        del R
+        ws_dev = [(p[0], p[1]), (p[2], p[3])]
+        st = status_word()
+        outs = gpu_quantize(ws_dev, cfg.T, st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        host = [(c.cpu().numpy(), s.cpu().numpy()) for c, s in outs]
+        for (wr, wi), (cn, sn) in zip(ws_dev, host):
+            check_quantized(wr.cpu().numpy(), wi.cpu().numpy(), cn, sn, cfg.T)
+        del p, ws_dev
+        outs_all += outs
+        host_all += host
+    for B in cfg.batches:
+        descs, xs = [], []
+        for i, spec in enumerate(cfg.layers):
+            xr, xi, xrn, xin = _x(cfg, i, B)
+            xs.append((xrn, xin))
+            (cu, su), (cw, sw) = outs_all[2 * i], outs_all[2 * i + 1]
+            descs.append(layer_desc(cu, su, cw, sw, xr, xi, spec.N, spec.K, B))
+        Q.ifq_gemv(descs, cfg.T, B)
+        torch.cuda.synchronize()
+        for i, (d, spec) in enumerate(zip(descs, cfg.layers)):
+            (cun, sun), (cwn, swn) = host_all[2 * i], host_all[2 * i + 1]
+            rows = sample_rows(spec.N, 128, rng)
+            check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cun, sun, cwn, swn, *xs[i], rows)
+
+
+# ---------------------------------------------------------------- edge cases
+def _rand_complex(rng, N, K, sigma=0.02):
+    return ((sigma * rng.standard_normal((N, K))).astype(np.float32),
+            (sigma * rng.standard_normal((N, K))).astype(np.float32))
+
+
+@pytest.mark.parametrize("N,K,T,conj", [(37, 64, 1, False), (129, 192, 3, True), (16, 320, 8, True),
+                                         (1, 64, 2, True), (300, 576, 2, False)])
+def test_ragged_shapes_all_batches(N, K, T, conj):
+    rng = np.random.default_rng(N * 1000 + K)
+    ws = [_rand_complex(rng, N, K)] + ([_rand_complex(rng, N, K, 0.03)] if conj else [])
+    ws_dev = [(to_dev(a), to_dev(b)) for a, b in ws]
+    outs = gpu_quantize(ws_dev, T)
+    torch.cuda.synchronize()
+    host = [(c.cpu().numpy(), s.cpu().numpy()) for c, s in outs]
+    for (wr, wi), (cn, sn) in zip(ws, host):
+        check_quantized(wr, wi, cn, sn, T)
+    cu, su = outs[0]
+    cw, sw = outs[1] if conj else (None, None)
+    cun, sun = host[0]
+    cwn, swn = host[1] if conj else (None, None)
+    for B in range(1, 17):
+        xr32 = rng.standard_normal((B, K)).astype(np.float32)
+        xi32 = rng.standard_normal((B, K)).astype(np.float32)
+        xr = torch.from_numpy(xr32).to(torch.bfloat16)
+        xi = torch.from_numpy(xi32).to(torch.bfloat16)
+        d = layer_desc(cu, su, cw, sw, xr.to(DEV), xi.to(DEV), N, K, B)
+        Q.ifq_gemv([d], T, B)
+        torch.cuda.synchronize()
+        check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cun, sun, cwn, swn,
+                      W.bf16_to_f32_numpy(xr), W.bf16_to_f32_numpy(xi))
+    for M in (1, 128, 131):
+        xr = torch.from_numpy(rng.standard_normal((M, K)).astype(np.float32)).to(torch.bfloat16)
+        xi = torch.from_numpy(rng.standard_normal((M, K)).astype(np.float32)).to(torch.bfloat16)
+        d = layer_desc(cu, su, cw, sw, xr.to(DEV), xi.to(DEV), N, K, M)
+        st = status_word()
+        Q.ifq_gemm([d], T, M, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cun, sun, cwn, swn,
+                      W.bf16_to_f32_numpy(xr), W.bf16_to_f32_numpy(xi))
+
+
+def test_quantizer_degenerate_inputs():
+    """All-zero weights, real-only weights, exact diagonal ties, signed zeros and non-finite entries."""
+    rng = np.random.default_rng(77)
+    N, K = 24, 64
+    zero = (np.zeros((N, K), np.float32), np.zeros((N, K), np.float32))
+    real_only = ((0.02 * rng.standard_normal((N, K))).astype(np.float32), np.zeros((N, K), np.float32))
+    ties_re = (0.01 * rng.integers(-3, 4, size=(N, K))).astype(np.float32)
+    ties_im = ties_re * rng.choice(np.array([1, -1], np.float32), size=(N, K))
+    ties = (ties_re, ties_im)
+    signed_zero = (np.where(rng.random((N, K)) < 0.5, -0.0, 0.0).astype(np.float32),
+                   np.where(rng.random((N, K)) < 0.5, -0.0, 0.0).astype(np.float32))
+    ws = [zero, real_only, ties, signed_zero]
+    ws_dev = [(to_dev(a), to_dev(b)) for a, b in ws]
+    st = status_word()
+    outs = gpu_quantize(ws_dev, 3, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for (wr, wi), (c, s) in zip(ws, outs):
+        check_quantized(wr, wi, c.cpu().numpy(), s.cpu().numpy(), 3)
+    assert np.all(outs[0][1].cpu().numpy() == 0)
+    # non-finite entries: quantized as 0, flagged
+    bad_re = (0.02 * rng.standard_normal((N, K))).astype(np.float32)
+    bad_im = (0.02 * rng.standard_normal((N, K))).astype(np.float32)
+    bad_re[3, 5], bad_im[7, 9], bad_re[0, 0] = np.nan, np.inf, -np.inf
+    st = status_word()
+    (c, s), = gpu_quantize([(to_dev(bad_re), to_dev(bad_im))], 2, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & Q.IFQ_DEV_NONFINITE
+    check_quantized(bad_re, bad_im, c.cpu().numpy(), s.cpu().numpy(), 2)
+
+
+def test_gemv_and_quantizer_are_bit_reproducible():
+    rng = np.random.default_rng(8)
+    N, K, T = 200, 1024, 2
+    ws_dev = [(to_dev(a), to_dev(b)) for a, b in (_rand_complex(rng, N, K), _rand_complex(rng, N, K))]
+    o1 = gpu_quantize(ws_dev, T)
+    o2 = gpu_quantize(ws_dev, T)
+    torch.cuda.synchronize()
+    for (c1, s1), (c2, s2) in zip(o1, o2):
+        assert torch.equal(c1, c2) and torch.equal(s1, s2)
+    xr = torch.from_numpy(rng.standard_normal((4, K)).astype(np.float32)).to(torch.bfloat16).to(DEV)
+    xi = torch.from_numpy(rng.standard_normal((4, K)).astype(np.float32)).to(torch.bfloat16).to(DEV)
+    d1 = layer_desc(o1[0][0], o1[0][1], o1[1][0], o1[1][1], xr, xi, N, K, 4)
+    d2 = layer_desc(o1[0][0], o1[0][1], o1[1][0], o1[1][1], xr, xi, N, K, 4)
+    Q.ifq_gemv([d1], T, 4)
+    Q.ifq_gemv([d2], T, 4)
+    m1 = layer_desc(o1[0][0], o1[0][1], o1[1][0], o1[1][1], xr, xi, N, K, 4)
+    m2 = layer_desc(o1[0][0], o1[0][1], o1[1][0], o1[1][1], xr, xi, N, K, 4)
+    Q.ifq_gemm([m1], T, 4)
+    Q.ifq_gemm([m2], T, 4)
+    torch.cuda.synchronize()
+    assert torch.equal(d1["y_re"], d2["y_re"]) and torch.equal(d1["y_im"], d2["y_im"])
+    assert torch.equal(m1["y_re"], m2["y_re"]) and torch.equal(m1["y_im"], m2["y_im"])
+
+
+def test_conversion_odd_width_and_subnormals():
+    rng = np.random.default_rng(9)
+    R = (0.02 * rng.standard_normal((10, 14))).astype(np.float32)   # m = 7: scalar path
+    R[0, 0], R[5, 7] = 1e-40, -3e-41
+    check_convert(R, gpu_convert(R))
+    R2 = (0.02 * rng.standard_normal((64, 128))).astype(np.float32)
+    R2[1, :4] = [1e-45, -1e-45, 2e-38, 0.0]
+    check_convert(R2, gpu_convert(R2))
