@@ -1,0 +1,538 @@
+"""Benchmark of the PhaseQuant / multiplication-free complex product path on B200.
+
+Default run (the contract line): one step is one pass of the whole path on the
+LLaMA-2-7B-shaped Fairy2i block (seven real layers q,k,v,o 4096x4096,
+gate,up 4096->11008, down 11008->4096; 2 residual stages; U and W):
+  1. widely-linear conversion of the seven real layers        (7 launches)
+  2. 2-stage PhaseQuant + pack of the 14 complex tensors      (1 memset + 2 launches)
+  3. L2 flush (256 MiB memset), then decode GEMV at B = 1     (1 launch, all 7 layers)
+  4. prefill GEMM at M = 2048 tokens                          (7 launches)
+Inputs are resident in HBM when the timed region starts; the metric value is
+the decode GEMV's algorithmic HBM bytes over its CUDA-event time; the prefill
+GEMM's equivalent TOP/s (8 M N K per stage and branch) is reported beside it.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  python bench.py --case gemv|gemm|quant|convert ...   (single-kernel cases for ncu)
+
+Multi-GPU (torchrun, one process per GPU): each rank runs an independent
+replica of the block (weak scaling, no data-path collective); timing is the
+max over ranks.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import bit_complex_quantized_b200 as Q  # noqa: E402
+from bit_complex_quantized_b200 import workloads as W  # noqa: E402
+
+METRIC = "decode GEMV HBM GB/s (% of peak); prefill GEMM equiv TOP/s at M=2048"
+WORKLOAD = "Fairy2i LLaMA-2-7B-shaped block (7 real layers -> 14 U/W tensors, 2 stages): conversion + " \
+           "PhaseQuant + decode GEMV B=1 + prefill GEMM M=2048"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ---------------------------------------------------------------- helpers
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def source_hash(name):
+    with open(os.path.join(ROOT, "bit_complex_quantized_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file, kernel, workload):
+    """dram bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel, {})
+    if e.get("source_sha256_16") != source_hash(kernel_file) or e.get("workload") != workload:
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- the block
+class Block:
+    """Device-resident state of the 7B-shaped block: real weights, planes, codes, activations."""
+
+    def __init__(self, dev, gemm_M=2048, decode_B=1):
+        self.cfg = W.config("c3")
+        self.cfg4 = W.config("c4")
+        self.T = self.cfg.T
+        self.dev = dev
+        self.R = []
+        self.planes = []
+        for i, spec in enumerate(self.cfg.layers):
+            self.R.append(torch.from_numpy(W.real_weight(self.cfg, i)).to(dev))
+            self.planes.append([torch.empty((spec.N, spec.K), dtype=torch.float32, device=dev) for _ in range(4)])
+        self.codes = []
+        for i, spec in enumerate(self.cfg.layers):
+            for _ in range(2):
+                self.codes.append((torch.empty((self.T, spec.N, spec.K // 4), dtype=torch.uint8, device=dev),
+                                   torch.empty((self.T, 2), dtype=torch.float32, device=dev)))
+        self.qt = []
+        for i in range(len(self.cfg.layers)):
+            p = self.planes[i]
+            self.qt.append((p[0], p[1], *self.codes[2 * i]))
+            self.qt.append((p[2], p[3], *self.codes[2 * i + 1]))
+        self.ws = torch.empty(Q.ifq_quantize_workspace_bytes(self.qt, self.T), dtype=torch.uint8, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.B, self.M = decode_B, gemm_M
+        self.gemv_layers = self._layers(self.cfg, self.B)
+        self.gemv_ws = torch.zeros(max(16, Q.ifq_gemv_workspace_bytes(self.gemv_layers, self.T, self.B)),
+                                   dtype=torch.uint8, device=dev)
+        self.gemm_layers = self._layers(self.cfg4, self.M)
+
+    def _layers(self, cfg, rows):
+        out = []
+        for i, spec in enumerate(cfg.layers):
+            xr, xi = W.activations(cfg, i, rows)
+            (cu, su), (cw, sw) = self.codes[2 * i], self.codes[2 * i + 1]
+            out.append(dict(codes_u=cu, scales_u=su, codes_w=cw, scales_w=sw, N=spec.N, K=spec.K,
+                            x_re=xr.to(self.dev), x_im=xi.to(self.dev),
+                            y_re=torch.empty((rows, spec.N), dtype=torch.float32, device=self.dev),
+                            y_im=torch.empty((rows, spec.N), dtype=torch.float32, device=self.dev)))
+        return out
+
+    # algorithmic bytes / flops
+    def convert_bytes(self):
+        return sum(32 * l.N * l.K for l in self.cfg.layers)
+
+    def quant_bytes(self):
+        # pass t reads w (8 B) and t earlier code bytes (t/4 B... per stage), writes 1/4 B, per complex entry
+        T = self.T
+        per_entry = 8 * T + sum(t / 4 for t in range(T)) + T / 4
+        return int(2 * sum(l.N * l.K for l in self.cfg.layers) * per_entry)
+
+    def gemv_bytes(self, B):
+        codes = W.code_bytes(self.cfg)
+        return codes + sum(4 * B * l.K + 8 * B * l.N for l in self.cfg.layers) + 2 * len(self.cfg.layers) * 8 * self.T
+
+    def gemm_flops(self):
+        return sum(8 * self.M * l.N * l.K * 2 * self.T for l in self.cfg.layers)
+
+    def step(self, ev=None):
+        s = torch.cuda.current_stream()
+        if ev:
+            ev[0].record(s)
+        for i in range(len(self.cfg.layers)):
+            Q.ifq_widely_linear_from_real(self.R[i], *self.planes[i])
+        if ev:
+            ev[1].record(s)
+        Q.ifq_quantize_pack(self.qt, self.T, self.ws, dev_status=self.status)
+        if ev:
+            ev[2].record(s)
+        self.flush.zero_()
+        if ev:
+            ev[3].record(s)
+        Q.ifq_gemv(self.gemv_layers, self.T, self.B, workspace=self.gemv_ws, dev_status=self.status)
+        if ev:
+            ev[4].record(s)
+        Q.ifq_gemm(self.gemm_layers, self.T, self.M, dev_status=self.status)
+        if ev:
+            ev[5].record(s)
+
+    def launches_per_step(self):
+        """Our kernels per step (the memsets are not counted): conversion, quantizer, GEMV, GEMM."""
+        gemv = 2 if self.B == 1 else 1  # B = 1: activation prep + integer product
+        return len(self.cfg.layers) + 2 + gemv + len(self.gemm_layers)
+
+
+def oracle_decode_sample(seconds_budget=10.0, rows_per_layer=64, max_reps=50):
+    """The fp64 oracle's decode product on a row sample of the block (CPU), in GB/s of codes.
+    Codes come from the C oracle's quantizer run on the same row sample (setup, untimed)."""
+    import oracle as O
+    from oracle import cref
+    cfg = W.config("c3")
+    rng = np.random.default_rng(123)
+    layers = []
+    for i, spec in enumerate(cfg.layers):
+        rows = np.sort(rng.choice(spec.N, size=rows_per_layer, replace=False))
+        R = W.real_weight(cfg, i)
+        n = spec.N
+        Rs = np.concatenate([R[rows], R[n + rows]], axis=0)
+        del R
+        ur, ui, wr, wi = O.widely_linear_planes_fp32(Rs)
+        cu, su = cref.quantize_tensor(ur, ui, cfg.T)
+        cw, sw = cref.quantize_tensor(wr, wi, cfg.T)
+        xr, xi = W.activations(cfg, i, 1)
+        layers.append((cu, su, cw, sw, W.bf16_to_f32_numpy(xr), W.bf16_to_f32_numpy(xi)))
+    nbytes = sum(2 * cfg.T * rows_per_layer * l.K // 4 for l in cfg.layers)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        for (cu, su, cw, sw, xr, xi) in layers:
+            O.product(cu, su, cw, sw, xr, xi)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds_budget or reps >= max_reps:
+            break
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        cores = 1
+    return {"value": nbytes * reps / el / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 NumPy oracle decode product, B=1, {rows_per_layer} sampled rows of each of the 7 "
+                      f"layers, U+W, T=2 ({nbytes / 1e6:.2f} MB of codes per rep), {reps} reps in {el:.1f} s"}
+
+
+# ---------------------------------------------------------------- e2e
+def e2e_decode(block, steps, warmup):
+    """Decode GEMV through the public API with host buffers: per step, pinned host -> device
+    copy of every layer's x, the grouped GEMV, device -> host copy of every y."""
+    dev = block.dev
+    host_x = [(L["x_re"].cpu().pin_memory(), L["x_im"].cpu().pin_memory()) for L in block.gemv_layers]
+    host_y = [(torch.empty_like(L["y_re"], device="cpu").pin_memory(),
+               torch.empty_like(L["y_im"], device="cpu").pin_memory()) for L in block.gemv_layers]
+    h2d = sum(a.numel() * a.element_size() + b.numel() * b.element_size() for a, b in host_x)
+    d2h = sum(a.numel() * a.element_size() + b.numel() * b.element_size() for a, b in host_y)
+
+    def one():
+        for L, (xr, xi) in zip(block.gemv_layers, host_x):
+            L["x_re"].copy_(xr, non_blocking=True)
+            L["x_im"].copy_(xi, non_blocking=True)
+        Q.ifq_gemv(block.gemv_layers, block.T, block.B, workspace=block.gemv_ws, dev_status=block.status)
+        for L, (yr, yi) in zip(block.gemv_layers, host_y):
+            yr.copy_(L["y_re"], non_blocking=True)
+            yi.copy_(L["y_im"], non_blocking=True)
+
+    times = []
+    for i in range(warmup + steps):
+        block.flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        one()
+        b.record()
+        torch.cuda.synchronize()
+        if i >= warmup:
+            times.append(a.elapsed_time(b) * 1e-3)
+    t = statistics.mean(times)
+    return {"value": block.gemv_bytes(block.B) / t / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": t * 1e3}
+
+
+# ---------------------------------------------------------------- main arm
+def run_ours(args):
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    block = Block(dev)
+    for _ in range(args.warmup):
+        block.step()
+    torch.cuda.synchronize()
+    assert int(block.status.item()) == 0, "device status set during warm-up"
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    clocks = Clocks(local)
+    clocks.start()
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for k in range(args.steps):
+        block.step(evs[k])
+    end.record()
+    torch.cuda.synchronize()
+    if ws > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    total_s = start.elapsed_time(end) * 1e-3
+    per = {name: statistics.mean(e[a].elapsed_time(e[b]) * 1e-3 for e in evs)
+           for name, a, b in (("convert", 0, 1), ("quant", 1, 2), ("gemv", 3, 4), ("gemm", 4, 5))}
+    assert int(block.status.item()) == 0, "device status set during timing"
+
+    # max over ranks of every time
+    vals = torch.tensor([total_s, per["convert"], per["quant"], per["gemv"], per["gemm"]], dtype=torch.float64,
+                        device=dev)
+    if ws > 1:
+        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
+    total_s, t_conv, t_quant, t_gemv, t_gemm = [float(v) for v in vals.cpu()]
+
+    pk, pk_src = peaks()
+    hbm = float(pk["hbm_gbs"])
+    tf_sus = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+    gemv_bytes = block.gemv_bytes(block.B)
+    gemv_gbs = gemv_bytes / t_gemv / 1e9
+    gemm_tops = block.gemm_flops() / t_gemm / 1e12
+    conv_gbs = block.convert_bytes() / t_conv / 1e9
+    quant_gbs = block.quant_bytes() / t_quant / 1e9
+    e2e = None
+    if rank == 0:
+        e2e = e2e_decode(block, steps=max(args.steps, 5), warmup=3)
+    cpu = None
+    if rank == 0 and ws == 1 and not args.skip_cpu_baseline:
+        cpu = oracle_decode_sample(seconds_budget=args.cpu_seconds)
+    if ws > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    kernels = {
+        "gemv": {"bound": "hbm", "achieved": gemv_gbs, "peak": hbm, "unit": "GB/s", "frac": gemv_gbs / hbm,
+                 "us": t_gemv * 1e6, "algorithmic_bytes": gemv_bytes,
+                 "traffic": recorded_traffic("gemv.cu", "gemv", "c3_b1")},
+        "gemm": {"bound": "tensor", "achieved": gemm_tops, "peak": tf_sus, "unit": "TFLOP/s",
+                 "frac": gemm_tops / tf_sus, "us": t_gemm * 1e6, "equiv_flops": block.gemm_flops(),
+                 "traffic": recorded_traffic("gemm.cu", "gemm", "c4_m2048")},
+        "quantize": {"bound": "hbm", "achieved": quant_gbs, "peak": hbm, "unit": "GB/s", "frac": quant_gbs / hbm,
+                     "us": t_quant * 1e6, "algorithmic_bytes": block.quant_bytes()},
+        "convert": {"bound": "hbm", "achieved": conv_gbs, "peak": hbm, "unit": "GB/s", "frac": conv_gbs / hbm,
+                    "us": t_conv * 1e6, "algorithmic_bytes": block.convert_bytes()},
+    }
+    dominant = max(("gemv", "gemm", "quantize", "convert"), key=lambda k: kernels[k]["us"])
+    rl = dict(kernels[dominant])
+    line = {
+        "metric": METRIC,
+        "value": ws * gemv_gbs,
+        "unit": "GB/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_s / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 activations x 2-bit codes, f32 accumulate; f64 scale reduction",
+        "data": "synthetic: seeded N(0,0.02) real weights, N(0,1) bf16 activations",
+        "config": {"workload": WORKLOAD, "decode_batch": block.B, "prefill_M": block.M, "stages": block.T,
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                   "l2": "256 MiB L2 flush before the GEMV in every step; conversion/quantizer inputs (1.6 GB) "
+                         "exceed L2"},
+        "prefill_gemm": {"value": ws * gemm_tops, "unit": "TOP/s (equivalent dense, 8 M N K per stage and branch)",
+                         "frac_of_sustained_bf16": gemm_tops / tf_sus},
+        "roofline": {"kernel": dominant, "bound": rl["bound"], "achieved": rl["achieved"], "peak": rl["peak"],
+                     "unit": rl["unit"], "frac": rl["frac"], "traffic": rl.get("traffic"),
+                     "peak_source": f"{pk_src} ({'bf16_tflops_sustained' if rl['bound'] == 'tensor' else 'hbm_gbs'})"},
+        "roofline_decode": {"kernel": "gemv", "bound": "hbm", "achieved": gemv_gbs, "peak": hbm, "unit": "GB/s",
+                            "frac": gemv_gbs / hbm, "traffic": kernels["gemv"]["traffic"],
+                            "peak_source": f"{pk_src} (hbm_gbs)"},
+        "kernels": kernels,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": block.launches_per_step() * args.steps,
+        "clocks": clk,
+    }
+    print(json.dumps(line))
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    reps = []
+    for i in range(args.warmup + args.steps):
+        r = oracle_decode_sample(seconds_budget=args.cpu_seconds / max(1, args.steps), rows_per_layer=32,
+                                 max_reps=5)
+        if i >= args.warmup:
+            reps.append(r)
+    v = statistics.mean(r["value"] for r in reps)
+    cpu = dict(reps[-1])
+    cpu["value"] = v
+    line = {"metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "decode_batch": 1, "stages": 2},
+            "cpu_baseline": cpu,
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+# ---------------------------------------------------------------- single-kernel cases (ncu)
+def run_case(args):
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    if args.case == "gemv":
+        # 70B-shaped layer set (321 MB of codes, larger than L2), random codes: the kernel's
+        # work does not depend on code values.
+        cfg = W.config("c5")
+        layers = []
+        for i, spec in enumerate(cfg.layers):
+            def rnd(shape):
+                return torch.randint(0, 256, shape, dtype=torch.uint8, device=dev, generator=g)
+            sc = lambda: torch.full((cfg.T, 2), 0.01, dtype=torch.float32, device=dev)  # noqa: E731
+            xr, xi = W.activations(cfg, i, args.batch)
+            layers.append(dict(codes_u=rnd((cfg.T, spec.N, spec.K // 4)), scales_u=sc(),
+                               codes_w=rnd((cfg.T, spec.N, spec.K // 4)), scales_w=sc(), N=spec.N, K=spec.K,
+                               x_re=xr.to(dev), x_im=xi.to(dev),
+                               y_re=torch.empty((args.batch, spec.N), device=dev),
+                               y_im=torch.empty((args.batch, spec.N), device=dev)))
+        nbytes = W.code_bytes(cfg)
+        gws = torch.zeros(max(16, Q.ifq_gemv_workspace_bytes(layers, cfg.T, args.batch)), dtype=torch.uint8,
+                          device=dev)
+
+        def fn():
+            Q.ifq_gemv(layers, cfg.T, args.batch, workspace=gws)
+        label = f"gemv c5 B={args.batch}"
+    elif args.case == "gemm":
+        cfg = W.config("c4")
+        spec = cfg.layers[4]  # gate: N = 5504, K = 2048
+        M = 2048
+
+        def rnd(shape):
+            return torch.randint(0, 256, shape, dtype=torch.uint8, device=dev, generator=g)
+        xr, xi = W.activations(cfg, 4, M)
+        L = dict(codes_u=rnd((2, spec.N, spec.K // 4)), scales_u=torch.full((2, 2), 0.01, device=dev),
+                 codes_w=rnd((2, spec.N, spec.K // 4)), scales_w=torch.full((2, 2), 0.01, device=dev),
+                 N=spec.N, K=spec.K, x_re=xr.to(dev), x_im=xi.to(dev),
+                 y_re=torch.empty((M, spec.N), device=dev), y_im=torch.empty((M, spec.N), device=dev))
+        nbytes = 8 * M * spec.N * spec.K * 4  # equiv flops
+
+        def fn():
+            Q.ifq_gemm([L], 2, M)
+        label = "gemm c4 gate M=2048"
+    elif args.case == "quant":
+        cfg = W.config("c3")
+        spec = cfg.layers[4]
+        ts = []
+        for _ in range(2):
+            wr = 0.02 * torch.randn((spec.N, spec.K), device=dev, generator=g)
+            wi = 0.02 * torch.randn((spec.N, spec.K), device=dev, generator=g)
+            ts.append((wr, wi, torch.empty((2, spec.N, spec.K // 4), dtype=torch.uint8, device=dev),
+                       torch.empty((2, 2), device=dev)))
+        wsb = torch.empty(Q.ifq_quantize_workspace_bytes(ts, 2), dtype=torch.uint8, device=dev)
+        nbytes = 2 * spec.N * spec.K * 16.75
+
+        def fn():
+            Q.ifq_quantize_pack(ts, 2, wsb)
+        label = "quantize c3 gate U+W T=2"
+    elif args.case == "convert":
+        cfg = W.config("c3")
+        spec = cfg.layers[4]
+        R = 0.02 * torch.randn(spec.real_shape, device=dev, generator=g)
+        planes = [torch.empty((spec.N, spec.K), device=dev) for _ in range(4)]
+        nbytes = 32 * spec.N * spec.K
+
+        def fn():
+            Q.ifq_widely_linear_from_real(R, *planes)
+        label = "convert c3 gate"
+    else:
+        raise SystemExit("unknown case")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b) * 1e-3)
+    t = statistics.median(times)
+    unit = "TOP/s" if args.case == "gemm" else "GB/s"
+    print(json.dumps({"case": label, "median_us": t * 1e6, "min_us": min(times) * 1e6,
+                      "rate": nbytes / t / (1e12 if args.case == "gemm" else 1e9), "unit": unit}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--case", choices=["gemv", "gemm", "quant", "convert"], default=None)
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    elif args.case:
+        run_case(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

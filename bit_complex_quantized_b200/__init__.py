@@ -15,6 +15,7 @@ from ._lib import (  # noqa: F401
     LIB_PATH,
     ifq_gemm,
     ifq_gemv,
+    ifq_gemv_workspace_bytes,
     ifq_quantize_pack,
     ifq_quantize_workspace_bytes,
     ifq_status_string,

@@ -24,6 +24,7 @@ EXPORTED = (
     "ifq_widely_linear_from_real",
     "ifq_quantize_workspace_bytes",
     "ifq_quantize_pack",
+    "ifq_gemv_workspace_bytes",
     "ifq_gemv",
     "ifq_gemm",
 )
@@ -72,8 +73,10 @@ def load():
     lib.ifq_quantize_workspace_bytes.argtypes = [ctypes.POINTER(QTensor), i32, i32]
     lib.ifq_quantize_pack.restype = i32
     lib.ifq_quantize_pack.argtypes = [ctypes.POINTER(QTensor), i32, i32, vp, sz, vp, vp]
+    lib.ifq_gemv_workspace_bytes.restype = sz
+    lib.ifq_gemv_workspace_bytes.argtypes = [ctypes.POINTER(Layer), i32, i32, i32]
     lib.ifq_gemv.restype = i32
-    lib.ifq_gemv.argtypes = [ctypes.POINTER(Layer), i32, i32, i32, vp, vp]
+    lib.ifq_gemv.argtypes = [ctypes.POINTER(Layer), i32, i32, i32, vp, sz, vp, vp]
     lib.ifq_gemm.restype = i32
     lib.ifq_gemm.argtypes = [ctypes.POINTER(Layer), i32, i32, i64, vp, vp]
     _lib = lib
@@ -139,10 +142,19 @@ def _layers(layers):
     return arr
 
 
-def ifq_gemv(layers, T, B, dev_status=None, stream=None):
+def ifq_gemv_workspace_bytes(layers, T, B):
+    return int(load().ifq_gemv_workspace_bytes(_layers(layers), len(layers), T, B))
+
+
+def ifq_gemv(layers, T, B, workspace=None, dev_status=None, stream=None, workspace_bytes=None):
     """layers: list of dicts with codes_u, scales_u, codes_w, scales_w (or None), N, K,
-    x_re, x_im (bf16 [B][K]), y_re, y_im (float32 [B][N])."""
-    _check(load().ifq_gemv(_layers(layers), len(layers), T, B, _ptr(dev_status), _stream(stream)))
+    x_re, x_im (bf16 [B][K]), y_re, y_im (float32 [B][N]).  workspace: a device
+    buffer of ifq_gemv_workspace_bytes() bytes, zero-filled before its first use."""
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if workspace_bytes is not None:
+        nbytes = workspace_bytes
+    _check(load().ifq_gemv(_layers(layers), len(layers), T, B, _ptr(workspace), nbytes, _ptr(dev_status),
+                           _stream(stream)))
 
 
 def ifq_gemm(layers, T, M, dev_status=None, stream=None):

@@ -1,0 +1,610 @@
+// Decode product for one token (B = 1) on the integer tensor cores, exactly
+// ("Fairy2i write-up" §2.1, §4.2; "iFairy article" §二.2; "iFairy talk notes" §2.3.1).
+//
+// Re-coding the 2-bit code.  With k = 2 s + c (c: axis bit, s: sign bit), the
+// real and imaginary parts of the codeword [1, i, -1, -i][k] are
+//     Br = (1-c)(1-2s),   Bi = c(1-2s),
+// which mix c and s.  In the Gray code g1 = s, g0 = c XOR s they become affine:
+//     Br = 1 - g0 - g1,   Bi = g0 - g1,
+// so two 0/1 bit-planes per code suffice:
+//     sum_j Br_j x_j = sum_j x_j - G0 - G1,   sum_j Bi_j x_j = G0 - G1,   G_b = sum_j g_b,j x_j.
+// In registers: gray = w ^ ((w >> 1) & 0x5555...), then one AND per (plane,
+// in-byte position q) selects 4 codes -- one per byte, all at position q -- as
+// int8 operands 4^q g0 or 2*4^q g1.  Each (plane, q) has its own int32
+// accumulator, so no shift is needed; the weights are undone exactly when the
+// accumulators are combined.
+//
+// Activations.  ifq_gemv first runs gemv_prep_kernel: per block of up to 2048
+// K positions, x (bf16, both planes) is scaled by 2^E with the block maximum in
+// [2^29, 2^30) and rounded to an integer v, whose four balanced base-256 digits
+// are the bytes of (v + 0x80808080) ^ 0x80808080.  The rounding error is at
+// most 2^-E per position, so sum_j(|e_re,j| + |e_im,j|) <= 2048 * 2^-E, below
+// 4e-6 of the block's largest |x| -- inside the 1e-5 tolerance for any x.
+// The digits are stored in MMA-fragment order with the exact block sums of v.
+//
+// Main kernel (programmatic dependent launch after the prep kernel): the codes
+// are cut into 1 KB chunks (16 rows x 256 K positions of one (stage, branch)
+// matrix), ordered tile by tile, and every warp of a persistent grid takes an
+// equal contiguous range of chunks (stream-K), so the load is balanced to one
+// chunk.  A warp walks its range in pieces (one tile, one matrix, one K block
+// at most), streams each piece's 16 code rows into a double-buffered shared
+// slot with cp.async.bulk (one row per lane, completion on an mbarrier), and
+// runs mma.sync m16n8k32 s8 (columns = plane x digit, exact int32
+// accumulation).  Per tile it keeps the float64 output sums in registers; a
+// tile split between warps leaves one partial per warp in the workspace, and
+// the last of them to arrive (atomic ticket) adds the partials in warp order
+// and writes y -- results do not depend on timing.
+#include "ifq_common.cuh"
+#include "ifq_internal.h"
+
+#include <mutex>
+
+namespace ifq {
+namespace {
+
+constexpr int kKBlock = 2048;                  // K positions per exponent block
+constexpr int kKsteps = kKBlock / 32;          // MMA k-steps per block (64)
+constexpr int kWarps = 4;                      // warps per CTA in the main kernel
+constexpr int kPieceChunks = 8;                // at most 8 chunks (256 K positions each) per piece: one K block
+constexpr int kSlotRow = 576;                  // bytes per code row in a slot (512 + 64 pad: conflict-free)
+constexpr int kSlotBytes = 16 * kSlotRow;      // one 16-row slot
+constexpr int kMainSmem = kWarps * 2 * kSlotBytes + kWarps * 2 * 8;
+constexpr int kPrepThreads = 256;
+
+struct I8Layer {
+  const uint8_t* codes[2];
+  const float* scales[2];
+  const uint16_t* x[2];
+  float* y[2];
+  uint4* frag;            // [blocks][8 chunks][32 lanes][4]: a lane's 8 k-step fragments of a chunk, contiguous
+  double* bsum;           // [blocks][2]
+  int* bexp;              // [blocks]
+  float* partials;        // [tiles][chunks per tile][16][2] (one slot per warp touching the tile)
+  unsigned int* tickets;  // [tiles]
+  int64_t N, K;
+  int64_t chunk_begin;    // first global chunk
+  int64_t prep_begin;     // first prep CTA
+  int32_t tiles;          // 16-row tiles
+  int32_t blocks;         // K blocks
+  int32_t nbranch;
+  int32_t nch;            // 256-wide K chunks per row
+};
+
+struct I8Params {
+  I8Layer L[IFQ_MAX_GROUP];
+  int64_t total_chunks;
+  int count;
+  int T;
+  uint32_t* status;
+};
+
+__device__ __forceinline__ void imma_16832(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                           uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t gray(uint32_t w) { return w ^ ((w >> 1) & 0x55555555u); }
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ int find_layer_by(const I8Params& p, int64_t idx, bool prep) {
+  int li = 0;
+  while (li + 1 < p.count && idx >= (prep ? p.L[li + 1].prep_begin : p.L[li + 1].chunk_begin)) ++li;
+  return li;
+}
+
+// ---------------------------------------------------------------- prep kernel
+// One CTA per (layer, K block): exponent, digit fragments, exact sums of v.
+// It also zeroes the layer's tile tickets for the main kernel.
+__global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(const __grid_constant__ I8Params p) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ __align__(16) uint16_t xs[2][kKBlock];
+  __shared__ unsigned int smax[kPrepThreads / 32];
+  __shared__ long long ssum[2][kPrepThreads / 32];
+
+  const int li = find_layer_by(p, blockIdx.x, true);
+  const I8Layer& L = p.L[li];
+  const int b = (int)(blockIdx.x - L.prep_begin);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (b == 0)
+    for (int t = tid; t < L.tiles; t += kPrepThreads) L.tickets[t] = 0u;
+
+  const int64_t k0 = (int64_t)b * kKBlock;
+  const int klen = (int)(L.K - k0 < kKBlock ? L.K - k0 : kKBlock);  // multiple of 64
+  const int nchunks = (klen + 255) >> 8;
+
+  unsigned int mx = 0;
+  for (int pl = 0; pl < 2; ++pl) {
+    const int idx = tid * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (idx < klen) v = __ldg(reinterpret_cast<const uint4*>(L.x[pl] + k0 + idx));
+    *reinterpret_cast<uint4*>(&xs[pl][idx]) = v;
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      mx = max(mx, wv[q] & 0x7FFFu);
+      mx = max(mx, (wv[q] >> 16) & 0x7FFFu);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) smax[warp] = mx;
+  __syncthreads();
+  mx = 0;
+#pragma unroll
+  for (int w = 0; w < kPrepThreads / 32; ++w) mx = max(mx, smax[w]);
+  const bool nonfinite = mx >= 0x7F80u;
+  int E = 0;  // max |x| * 2^E in [2^29, 2^30)
+  if (mx != 0 && !nonfinite) {
+    const uint32_t f = mx << 16;
+    const int e = (f >> 23) ? (int)(f >> 23) - 127 : (31 - __clz(f)) - 149;
+    E = 29 - e;
+  }
+  if (nonfinite && tid == 0) set_status(p.status, IFQ_DEV_NONFINITE);
+  const int E1 = min(E, 127);
+  const float f1 = __int_as_float((E1 + 127) << 23);
+  const float f2 = __int_as_float((E - E1 + 127) << 23);
+
+  // Item (plane pl, in-byte position q, 16-position group grp = (chunk c, slice tq, word w))
+  // covers positions grp*16 + 4i + q, i = 0..3: bytes i of the code word w at position q.
+  long long vsum = 0;
+  const int nitems = nchunks * 128;
+  for (int it = tid; it < nitems; it += kPrepThreads) {
+    const int pl = it & 1, q = (it >> 1) & 3, grp = it >> 3;
+    uint32_t D[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = grp * 16 + 4 * i + q;
+      int v = 0;
+      if (j < klen && !nonfinite) {
+        const float xf = __uint_as_float((uint32_t)xs[pl][j] << 16);
+        v = __float2int_rn((xf * f1) * f2);
+      }
+      vsum += v;
+      D[i] = ((uint32_t)v + 0x80808080u) ^ 0x80808080u;
+    }
+    const uint32_t lo01 = __byte_perm(D[0], D[1], 0x5140), lo23 = __byte_perm(D[2], D[3], 0x5140);
+    const uint32_t hi01 = __byte_perm(D[0], D[1], 0x7362), hi23 = __byte_perm(D[2], D[3], 0x7362);
+    const uint32_t dig[4] = {__byte_perm(lo01, lo23, 0x5410), __byte_perm(lo01, lo23, 0x7632),
+                             __byte_perm(hi01, hi23, 0x5410), __byte_perm(hi01, hi23, 0x7632)};
+    const int c = grp >> 4, tqs = (grp >> 2) & 3, w = grp & 3;
+    const int ks = (w >> 1) * 4 + q;  // k-step within the chunk: (word pair, position)
+    // a lane's fragments for chunk c: 8 k-steps x (b0, b1) = 64 contiguous bytes
+    uint32_t* fr = reinterpret_cast<uint32_t*>(L.frag + ((int64_t)b * 8 + c) * 32 * 4) + ks * 2 + (w & 1);
+#pragma unroll
+    for (int d = 0; d < 4; ++d) fr[((pl * 4 + d) * 4 + tqs) * 16] = dig[d];
+  }
+#pragma unroll
+  for (int o = 16; o > 1; o >>= 1) vsum += __shfl_xor_sync(0xffffffffu, vsum, o);  // even / odd lanes
+  if (lane < 2) ssum[lane][warp] = vsum;
+  __syncthreads();
+  if (tid < 2) {
+    long long s = 0;
+#pragma unroll
+    for (int w = 0; w < kPrepThreads / 32; ++w) s += ssum[tid][w];
+    L.bsum[2 * b + tid] = nonfinite ? __longlong_as_double(0x7FF8000000000000LL) : (double)s;
+    if (tid == 0) L.bexp[b] = E;
+  }
+}
+
+// ---------------------------------------------------------------- main kernel
+// A piece: chunks [ch, ch + len) of one (tile, matrix) row block, inside one K block.
+struct Piece {
+  int li;
+  int mat;
+  int ch;
+  int len;
+  int64_t tile;
+  int64_t gbegin;  // global index of its first chunk
+};
+
+__device__ __forceinline__ int piece_len(const I8Layer& L, int ch, int64_t gbegin, int64_t c_hi) {
+  const int block_end = min(L.nch, (ch / 8 + 1) * 8);
+  int64_t len = min(block_end - ch, kPieceChunks);
+  if (gbegin + len > c_hi) len = c_hi - gbegin;
+  return (int)len;
+}
+
+// The piece that starts at global chunk c (one division chain per warp, at its start).
+__device__ __forceinline__ Piece make_piece(const I8Params& p, int64_t c, int64_t c_hi) {
+  Piece pc;
+  pc.li = find_layer_by(p, c, false);
+  const I8Layer& L = p.L[pc.li];
+  const int64_t tc = (int64_t)p.T * L.nbranch * L.nch;  // chunks per tile
+  const int64_t local = c - L.chunk_begin;
+  pc.tile = local / tc;
+  const int r = (int)(local - pc.tile * tc);
+  pc.mat = r / L.nch;
+  pc.ch = r - pc.mat * L.nch;
+  pc.gbegin = c;
+  pc.len = piece_len(L, pc.ch, c, c_hi);
+  return pc;
+}
+
+// The piece after `pc` in chunk order (chunks, then matrices, then tiles, then layers).
+__device__ __forceinline__ Piece next_piece(const I8Params& p, const Piece& pc, int64_t c_hi) {
+  Piece n = pc;
+  n.gbegin = pc.gbegin + pc.len;
+  n.ch = pc.ch + pc.len;
+  const I8Layer* L = &p.L[n.li];
+  if (n.ch >= L->nch) {
+    n.ch = 0;
+    if (++n.mat >= p.T * L->nbranch) {
+      n.mat = 0;
+      if (++n.tile >= L->tiles) {
+        n.tile = 0;
+        ++n.li;
+        L = &p.L[n.li];
+      }
+    }
+  }
+  n.len = piece_len(*L, n.ch, n.gbegin, c_hi);
+  return n;
+}
+
+// Warp w < W owns chunks [lo(w), lo(w+1)) with lo(w) = floor(w C / W); W <= C.
+__device__ __forceinline__ int64_t range_lo(int64_t w, int64_t C, int64_t W) { return (w * C) / W; }
+
+__device__ __forceinline__ int64_t warp_of_chunk(int64_t c, int64_t C, int64_t W) {
+  int64_t w = (c * W) / C;
+  while (w + 1 < W && range_lo(w + 1, C, W) <= c) ++w;
+  while (w > 0 && range_lo(w, C, W) > c) --w;
+  return w;
+}
+
+// Lanes 0..15 each copy one code row of the piece into the slot.
+__device__ __forceinline__ void issue_piece(const I8Params& p, const Piece& pc, uint32_t slot, uint64_t* bar,
+                                            int lane) {
+  const I8Layer& L = p.L[pc.li];
+  const int64_t row0 = pc.tile * 16;
+  const int rows = (int)(L.N - row0 < 16 ? L.N - row0 : 16);
+  const int64_t kend = (int64_t)(pc.ch + pc.len) * 256 < L.K ? (int64_t)(pc.ch + pc.len) * 256 : L.K;
+  const uint32_t bytes = (uint32_t)((kend - (int64_t)pc.ch * 256) >> 2);
+  if (lane == 0) mbar_arrive_expect_tx(bar, bytes * (uint32_t)rows);
+  __syncwarp();
+  if (lane < rows) {
+    const int t = pc.mat / L.nbranch, br = pc.mat % L.nbranch;
+    const int64_t rb = L.K >> 2;
+    const uint8_t* src = L.codes[br] + ((int64_t)t * L.N + row0 + lane) * rb + (int64_t)pc.ch * 64;
+    bulk_g2s(slot + lane * kSlotRow, src, bytes, bar);
+  }
+}
+
+__global__ void __launch_bounds__(kWarps * 32, 3) gemv_i8_kernel(const __grid_constant__ I8Params p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, tq = lane & 3;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * 2 * kSlotBytes) + warp * 2;
+  const uint32_t slots = smem_u32(smem + warp * 2 * kSlotBytes);
+  if (lane == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  // W <= C warps take part, so every range is non-empty and the warps owning a
+  // tile's chunks are consecutive.
+  const int64_t C = p.total_chunks;
+  const int64_t W = (int64_t)gridDim.x * kWarps < C ? (int64_t)gridDim.x * kWarps : C;
+  const int64_t gw = (int64_t)blockIdx.x * kWarps + warp;
+  if (gw >= W) return;
+  const int64_t c_lo = range_lo(gw, C, W), c_hi = range_lo(gw + 1, C, W);
+
+  int abort_flag = 0;
+  uint32_t phases = 0u;  // bit s: parity of the next completion of slot s
+  int s = 0;
+  // The code bytes do not depend on the prep kernel: start streaming them, then
+  // wait for the prep kernel's activation digits.
+  Piece cur = make_piece(p, c_lo, c_hi);
+  issue_piece(p, cur, slots, &bars[0], lane);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  double yr[2] = {0.0, 0.0}, yi[2] = {0.0, 0.0};  // rows g, g+8 of the current tile (tq == 0)
+  int acc0[4][4], acc1[4][4];  // [position q][fragment reg], summed over the pieces of one (tile, matrix, K block)
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) acc0[q][r] = acc1[q][r] = 0;
+  bool first_of_block = (cur.ch & 7) == 0;  // this (tile, matrix, block) run starts the block
+
+  for (;;) {
+    const int64_t nc = cur.gbegin + cur.len;
+    const bool has_next = nc < c_hi;
+    Piece nxt;
+    if (has_next) {
+      nxt = next_piece(p, cur, c_hi);
+      issue_piece(p, nxt, slots + (s ^ 1) * kSlotBytes, &bars[s ^ 1], lane);
+    }
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait_bounded_sleep(&bars[s], (phases >> s) & 1u, &abort_flag);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    phases ^= 1u << s;
+    if (!ok) {
+      if (lane == 0) set_status(p.status, IFQ_DEV_TIMEOUT);
+      if (has_next) {  // let the other slot's copies land before leaving
+        volatile int never = 0;
+        if (lane == 0) mbar_wait_bounded(&bars[s ^ 1], (phases >> (s ^ 1)) & 1u, &never);
+      }
+      return;
+    }
+
+    const I8Layer& L = p.L[cur.li];
+    const uint32_t slot = slots + s * kSlotBytes;
+    const int blk = cur.ch >> 3;
+    // fragments of this piece's first chunk for this lane; 32 lanes x 64 B per chunk
+    const uint4* fr = L.frag + (((int64_t)blk * 8 + (cur.ch & 7)) * 32 + lane) * 4;
+    const uint32_t rowa = slot + g * kSlotRow + tq * 16, rowb = rowa + 8 * kSlotRow;
+
+    // Positions past K carry zero activation digits, so code bytes there (stale or not) add nothing.
+    // The next chunk's code words and fragments are loaded while this chunk computes.
+    uint4 va = lds128(rowa), vb = lds128(rowb);
+    uint4 F[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) F[k] = __ldg(fr + k);
+    for (int c = 0; c < cur.len; ++c) {
+      uint4 nva = va, nvb = vb, NF[4];
+      const int cn = c + 1 < cur.len ? c + 1 : c;
+      nva = lds128(rowa + cn * 64);
+      nvb = lds128(rowb + cn * 64);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) NF[k] = __ldg(fr + cn * 128 + k);
+#pragma unroll
+      for (int wp = 0; wp < 2; ++wp) {
+        const uint32_t a0 = gray(wp ? va.z : va.x), a1 = gray(wp ? va.w : va.y);
+        const uint32_t b0 = gray(wp ? vb.z : vb.x), b1 = gray(wp ? vb.w : vb.y);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int ks = wp * 4 + q;
+          const uint32_t fx = (ks & 1) ? F[ks >> 1].z : F[ks >> 1].x;
+          const uint32_t fy = (ks & 1) ? F[ks >> 1].w : F[ks >> 1].y;
+          const uint32_t m0 = 0x01010101u << (2 * q), m1 = 0x02020202u << (2 * q);
+          imma_16832(acc0[q], a0 & m0, b0 & m0, a1 & m0, b1 & m0, fx, fy);
+          imma_16832(acc1[q], a0 & m1, b0 & m1, a1 & m1, b1 & m1, fx, fy);
+        }
+      }
+      va = nva;
+      vb = nvb;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) F[k] = NF[k];
+    }
+    __syncwarp();  // every lane is done with this slot before it is refilled
+
+    // The int32 sums stay open while the next piece continues the same (tile, matrix, K block).
+    const bool same_run = has_next && nxt.li == cur.li && nxt.tile == cur.tile && nxt.mat == cur.mat &&
+                          (nxt.ch >> 3) == blk;
+    if (!same_run) {
+    // ---- combine: weights 4^q (g0) and 2*4^q, -128 at q = 3 (g1) -> 64 G0 and 128 G1, exact int32
+    double qa[2], qb[2];  // rows g, g+8: this thread's two digit columns, combined
+    {
+      int G0[4], G1[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        G0[r] = 64 * acc0[0][r] + 16 * acc0[1][r] + 4 * acc0[2][r] + acc0[3][r];
+        G1[r] = 64 * acc1[0][r] + 16 * acc1[1][r] + 4 * acc1[2][r] - acc1[3][r];
+      }
+      const double dscale = (tq & 1) ? 65536.0 : 1.0;  // columns 2tq, 2tq+1 hold digits 2(tq&1), +1
+      qa[0] = dscale * ((double)G0[0] + 256.0 * (double)G0[1]);
+      qa[1] = dscale * ((double)G0[2] + 256.0 * (double)G0[3]);
+      qb[0] = dscale * ((double)G1[0] + 256.0 * (double)G1[1]);
+      qb[1] = dscale * ((double)G1[2] + 256.0 * (double)G1[3]);
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      qa[r] += __shfl_xor_sync(0xffffffffu, qa[r], 1);
+      qb[r] += __shfl_xor_sync(0xffffffffu, qb[r], 1);
+    }
+    double oa[2], ob[2];  // threads tq 0,1 hold plane re, 2,3 plane im: fetch the other plane
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      oa[r] = __shfl_xor_sync(0xffffffffu, qa[r], 2);
+      ob[r] = __shfl_xor_sync(0xffffffffu, qb[r], 2);
+    }
+    if (tq == 0) {
+      const int t = cur.mat / L.nbranch, br = cur.mat % L.nbranch;
+      const double sr = (double)__ldg(L.scales[br] + 2 * t), si = (double)__ldg(L.scales[br] + 2 * t + 1);
+      // the block sums of v count the whole block; a piece covers part of it, so use the
+      // sums only once per (tile, matrix, block): on the piece that starts the block's first chunk
+      const double inv = __longlong_as_double((long long)(1023 - L.bexp[blk]) << 52);  // 2^-E
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        // G0 = QA / 64, G1 = QB / 128;  P_r = S - G0 - G1,  P_i = G0 - G1 (S added by the block's first piece)
+        const double Prr = -qa[r] * 0.015625 - qb[r] * 0.0078125;
+        const double Pir = qa[r] * 0.015625 - qb[r] * 0.0078125;
+        const double Pri = -oa[r] * 0.015625 - ob[r] * 0.0078125;
+        const double Pii = oa[r] * 0.015625 - ob[r] * 0.0078125;
+        double pr = 0.0, pi = 0.0;
+        if (first_of_block) {
+          pr = L.bsum[2 * blk];
+          pi = L.bsum[2 * blk + 1];
+        }
+        double vr, vi;
+        if (br == 0) {
+          vr = sr * (Prr + pr) - si * Pii;
+          vi = sr * (Pri + pi) + si * Pir;
+        } else {
+          vr = sr * (Prr + pr) + si * Pii;
+          vi = si * Pir - sr * (Pri + pi);
+        }
+        yr[r] += vr * inv;
+        yi[r] += vi * inv;
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) acc0[q][r] = acc1[q][r] = 0;
+    first_of_block = has_next && (nxt.ch & 7) == 0;
+    }  // !same_run
+
+    // ---- tile finished for this warp: write y, or a partial and possibly reduce
+    const bool tile_done = !has_next || nxt.li != cur.li || nxt.tile != cur.tile;
+    if (tile_done) {
+      const int64_t tc = (int64_t)p.T * L.nbranch * L.nch;
+      const int64_t tb = L.chunk_begin + cur.tile * tc;
+      const int64_t w_first = warp_of_chunk(tb, C, W), w_last = warp_of_chunk(tb + tc - 1, C, W);
+      const int nparts = (int)(w_last - w_first + 1);
+      const int64_t row0 = cur.tile * 16;
+      if (nparts == 1) {
+        if (tq == 0) {
+#pragma unroll
+          for (int r = 0; r < 2; ++r)
+            if (row0 + g + 8 * r < L.N) {
+              L.y[0][row0 + g + 8 * r] = (float)yr[r];
+              L.y[1][row0 + g + 8 * r] = (float)yi[r];
+            }
+        }
+      } else {
+        float* part = L.partials + (cur.tile * tc + (gw - w_first)) * 32;
+        if (tq == 0) {
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            part[2 * (g + 8 * r)] = (float)yr[r];
+            part[2 * (g + 8 * r) + 1] = (float)yi[r];
+          }
+        }
+        __threadfence();
+        __syncwarp();
+        unsigned prev = 0;
+        if (lane == 0) prev = atomicAdd(L.tickets + cur.tile, 1u);
+        prev = __shfl_sync(0xffffffffu, prev, 0);
+        if (prev == (unsigned)(nparts - 1)) {
+          __threadfence();
+          if (lane < 16 && row0 + lane < L.N) {
+            const float* pt = L.partials + cur.tile * tc * 32 + 2 * lane;
+            float ar = 0.0f, ai = 0.0f;
+            for (int k = 0; k < nparts; ++k) {
+              ar += __ldcg(pt + k * 32);
+              ai += __ldcg(pt + k * 32 + 1);
+            }
+            L.y[0][row0 + lane] = ar;
+            L.y[1][row0 + lane] = ai;
+          }
+          if (lane == 0) L.tickets[cur.tile] = 0u;
+        }
+      }
+      yr[0] = yr[1] = yi[0] = yi[1] = 0.0;
+    }
+    if (!has_next) break;
+    cur = nxt;
+    s ^= 1;
+  }
+}
+
+// Workspace layout: 256 B header (unused), then per layer, each region
+// 256-byte aligned: fragments, block sums, block exponents, partials, tickets.
+struct WsLayout {
+  size_t frag, bsum, bexp, part, tick;
+};
+
+inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+size_t layout_layers(const ifq_layer* Ls, int count, int T, WsLayout* out) {
+  size_t off = 256;
+  for (int i = 0; i < count; ++i) {
+    const int64_t tiles = (Ls[i].N + 15) / 16;
+    const int64_t blocks = (Ls[i].K + kKBlock - 1) / kKBlock;
+    const int64_t nmat = (int64_t)T * (Ls[i].codes_w ? 2 : 1);
+    WsLayout w;
+    w.frag = off;
+    off = align256(off + (size_t)blocks * 8 * 32 * 64);
+    w.bsum = off;
+    off = align256(off + (size_t)blocks * 16);
+    w.bexp = off;
+    off = align256(off + (size_t)blocks * 4);
+    const int64_t nch = (Ls[i].K + 255) / 256;
+    w.part = off;
+    off = align256(off + (size_t)tiles * nmat * nch * 32 * 4);
+    w.tick = off;
+    off = align256(off + (size_t)tiles * 4);
+    if (out) out[i] = w;
+  }
+  return off;
+}
+
+}  // namespace
+
+size_t gemv_i8_workspace_bytes(const ifq_layer* Ls, int count, int T) { return layout_layers(Ls, count, T, nullptr); }
+
+cudaError_t launch_gemv_i8(const ifq_layer* Ls, int count, int T, void* ws, uint32_t* dev_status, cudaStream_t s) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(gemv_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMainSmem);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  I8Params p;
+  memset(&p, 0, sizeof(p));
+  p.count = count;
+  p.T = T;
+  p.status = dev_status;
+  WsLayout lay[IFQ_MAX_GROUP];
+  layout_layers(Ls, count, T, lay);
+  char* base = static_cast<char*>(ws);
+  int64_t chunks = 0, preps = 0;
+  for (int i = 0; i < count; ++i) {
+    I8Layer& a = p.L[i];
+    a.codes[0] = Ls[i].codes_u;
+    a.scales[0] = Ls[i].scales_u;
+    a.codes[1] = Ls[i].codes_w;
+    a.scales[1] = Ls[i].scales_w;
+    a.nbranch = Ls[i].codes_w ? 2 : 1;
+    a.x[0] = Ls[i].x_re;
+    a.x[1] = Ls[i].x_im;
+    a.y[0] = Ls[i].y_re;
+    a.y[1] = Ls[i].y_im;
+    a.N = Ls[i].N;
+    a.K = Ls[i].K;
+    a.tiles = (int32_t)((a.N + 15) / 16);
+    a.blocks = (int32_t)((a.K + kKBlock - 1) / kKBlock);
+    a.frag = reinterpret_cast<uint4*>(base + lay[i].frag);
+    a.bsum = reinterpret_cast<double*>(base + lay[i].bsum);
+    a.bexp = reinterpret_cast<int*>(base + lay[i].bexp);
+    a.partials = reinterpret_cast<float*>(base + lay[i].part);
+    a.tickets = reinterpret_cast<unsigned int*>(base + lay[i].tick);
+    a.nch = (int32_t)((a.K + 255) / 256);
+    a.chunk_begin = chunks;
+    a.prep_begin = preps;
+    chunks += (int64_t)a.tiles * T * a.nbranch * a.nch;
+    preps += a.blocks;
+  }
+  p.total_chunks = chunks;
+  if (chunks >= ((int64_t)1 << 40) || preps > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+
+  gemv_prep_kernel<<<(unsigned)preps, kPrepThreads, 0, s>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t ctas = (int64_t)sms * 3;
+  const int64_t need = (chunks + kWarps - 1) / kWarps;  // at least one chunk per warp
+  if (ctas > need) ctas = need;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)ctas);
+  cfg.blockDim = dim3(kWarps * 32);
+  cfg.dynamicSmemBytes = kMainSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemv_i8_kernel, p);
+}
+
+}  // namespace ifq

@@ -59,10 +59,40 @@ IFQ_DEVINL bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that may suspend the thread for up to `hint_ns` while the phase is incomplete.
+IFQ_DEVINL bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 IFQ_DEVINL uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
   return t;
+}
+
+// As mbar_wait_bounded, but the waiting thread sleeps in the barrier between
+// polls instead of spinning, and reads the clock only every 64 polls (for
+// waits on copies that take microseconds).
+IFQ_DEVINL bool mbar_wait_bounded_sleep(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if ((i & 63u) == 0u) {
+      if (*abort) return false;
+      if (global_ns() - t0 > IFQ_WAIT_LIMIT_NS) {
+        *abort = 1;
+        return false;
+      }
+    }
+  }
 }
 
 // Waits until the phase with the given parity has completed.  Gives up and

@@ -19,6 +19,10 @@ cudaError_t launch_quantize(const ifq_qtensor* t, int count, int T, void* ws, ui
 
 cudaError_t launch_gemv(const ifq_layer* L, int count, int T, int B, uint32_t* dev_status, cudaStream_t s);
 
+// B = 1 integer tensor-core path (gemv_i8.cu) and its workspace size.
+size_t gemv_i8_workspace_bytes(const ifq_layer* L, int count, int T);
+cudaError_t launch_gemv_i8(const ifq_layer* L, int count, int T, void* ws, uint32_t* dev_status, cudaStream_t s);
+
 cudaError_t launch_gemm(const ifq_layer* L, int count, int T, int64_t M, uint32_t* dev_status, cudaStream_t s);
 
 }  // namespace ifq

@@ -53,15 +53,29 @@ struct QParams {
   uint32_t* status;
 };
 
-// Sector of w = a + ib: 0 -> 1, 1 -> i, 2 -> -1, 3 -> -i.  Ties on a diagonal go
-// counter-clockwise, w = 0 -> 0.  Exact in any IEEE precision the inputs fit.
+// Sector of w = a + ib as (cls, sgn) with k = 2 sgn + cls: 0 -> 1, 1 -> i,
+// 2 -> -1, 3 -> -i.  Written without branches for finite a, b in any IEEE
+// precision:
+//   |b| > |a|                       -> cls 1, sign of b
+//   |a| > |b|                       -> cls 0, sign of a
+//   |a| = |b| > 0 (a diagonal tie)  -> the sector counter-clockwise of it:
+//                                      cls 1 iff a, b have the same sign
+//   a = b = 0                       -> k = 0
+// (the four tie cases: 45 deg -> 1, 135 deg -> 2, -135 deg -> 3, -45 deg -> 0).
 template <typename F>
-__device__ __forceinline__ uint32_t phase_sector(F a, F b) {
+__device__ __forceinline__ uint32_t sector_code(F a, F b) {
   const F aa = fabs(a), ab = fabs(b);
-  if (b > aa || (a == b && b > F(0))) return 1u;
-  if (-a > ab || (b == -a && a < F(0))) return 2u;
-  if (-b > aa || (a == b && b < F(0))) return 3u;
-  return 0u;
+  const bool tie_same = (aa == ab) && (aa > F(0)) && ((a > F(0)) == (b > F(0)));
+  const uint32_t cls = (ab > aa) || tie_same;
+  const uint32_t sgn = cls ? (b < F(0)) : (a < F(0));
+  return 2u * sgn + cls;
+}
+
+// Exact reference form of the same rule, used for entries with a non-finite part
+// (taken as 0) on the rare slow path.
+__device__ __forceinline__ uint32_t sector_code_checked(float a, float b) {
+  if (!(isfinite(a) && isfinite(b))) return 0u;
+  return sector_code(a, b);
 }
 
 __device__ __forceinline__ double warp_sum(double v) {
@@ -100,87 +114,93 @@ __device__ __forceinline__ void block_sum3(double& a, double& b, unsigned long l
   __syncthreads();
 }
 
-template <bool FIRST>
+// One quad (4 weights -> one code byte) of stage PREV (0-based), given the
+// earlier stages' code bytes of the quad.  Residual entries are rebuilt in
+// float64 one earlier stage at a time: Re r -= s_re Br, Im r -= s_im Bi, i.e.
+// add -s or +s when the code is on that axis.  Accumulates the quad's class
+// sums; returns the code byte.
+template <int PREV>
+__device__ __forceinline__ uint32_t quad_code(const float (&wr)[4], const float (&wi)[4], const uint32_t (&prev)[8],
+                                              const double (&sr)[8], const double (&si)[8], bool checked,
+                                              double& S_re, double& S_im) {
+  uint32_t byte = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const bool fin = !checked || (isfinite(wr[e]) && isfinite(wi[e]));
+    uint32_t k;
+    if (PREV == 0) {
+      const float a = fin ? wr[e] : 0.0f, b = fin ? wi[e] : 0.0f;
+      k = sector_code(a, b);
+      const double v = (double)((k & 1u) ? fabsf(b) : fabsf(a));
+      if (k & 1u) S_im += v; else S_re += v;
+    } else {
+      double a = fin ? (double)wr[e] : 0.0, b = fin ? (double)wi[e] : 0.0;
+#pragma unroll
+      for (int u = 0; u < PREV; ++u) {
+        const uint32_t ku = (prev[u] >> (2 * e)) & 3u;
+        const double step_r = (ku & 2u) ? sr[u] : -sr[u];  // -s_re * Br for Br = +-1
+        const double step_i = (ku & 2u) ? si[u] : -si[u];
+        a = (ku & 1u) ? a : a + step_r;
+        b = (ku & 1u) ? b + step_i : b;
+      }
+      k = sector_code(a, b);
+      const double v = (k & 1u) ? fabs(b) : fabs(a);
+      if (k & 1u) S_im += v; else S_re += v;
+    }
+    byte |= k << (2 * e);
+  }
+  return byte;
+}
+
+template <int PREV>
 __global__ void __launch_bounds__(kQThreads) quant_stage_kernel(const __grid_constant__ QParams p) {
   // Find this block's tensor (at most IFQ_MAX_GROUP entries, uniform per block).
   int ti = 0;
   while (ti + 1 < p.count && (int64_t)blockIdx.x >= p.t[ti + 1].block_begin) ++ti;
   const QTensorArg& T = p.t[ti];
-  const int stage = p.stage;
   const int64_t blk = (int64_t)blockIdx.x - T.block_begin;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t quad0 = blk * kQuadsPerBlock + (int64_t)warp * (32 * kQuadsPerThread) + lane;
 
-  double s_prev_re[IFQ_MAX_STAGES], s_prev_im[IFQ_MAX_STAGES];
-  if (!FIRST) {
+  double sr[8], si[8];
 #pragma unroll
-    for (int u = 0; u < IFQ_MAX_STAGES; ++u) {
-      if (u < stage) {
-        s_prev_re[u] = (double)__ldg(T.scales + 2 * u);
-        s_prev_im[u] = (double)__ldg(T.scales + 2 * u + 1);
-      }
-    }
+  for (int u = 0; u < 8; ++u) {
+    sr[u] = u < PREV ? (double)__ldg(T.scales + 2 * u) : 0.0;
+    si[u] = u < PREV ? (double)__ldg(T.scales + 2 * u + 1) : 0.0;
   }
+
+  // Load all four quads first (8 x 128-bit weight loads, PREV byte loads each).
+  float wr[kQuadsPerThread][4], wi[kQuadsPerThread][4];
+  uint32_t prev[kQuadsPerThread][8];
+#pragma unroll
+  for (int q = 0; q < kQuadsPerThread; ++q) {
+    const int64_t quad = quad0 + 32 * q;
+    const bool ok = quad < T.nquads;
+    const float4 vr = ok ? __ldcs(reinterpret_cast<const float4*>(T.w_re) + quad) : make_float4(0, 0, 0, 0);
+    const float4 vi = ok ? __ldcs(reinterpret_cast<const float4*>(T.w_im) + quad) : make_float4(0, 0, 0, 0);
+    wr[q][0] = vr.x; wr[q][1] = vr.y; wr[q][2] = vr.z; wr[q][3] = vr.w;
+    wi[q][0] = vi.x; wi[q][1] = vi.y; wi[q][2] = vi.z; wi[q][3] = vi.w;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) prev[q][u] = (u < PREV && ok) ? __ldg(T.codes + (int64_t)u * T.nquads + quad) : 0u;
+  }
+
+  // Non-finite weights are rare: one check for all 16 entries, exact handling only then.
+  float z = 0.0f;
+#pragma unroll
+  for (int q = 0; q < kQuadsPerThread; ++q)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) z += wr[q][e] * 0.0f + wi[q][e] * 0.0f;
+  const bool bad = z != 0.0f;  // NaN iff some entry is NaN or infinite
 
   double S_re = 0.0, S_im = 0.0;
   unsigned long long C_re = 0;
-  int bad = 0;
-
 #pragma unroll
   for (int q = 0; q < kQuadsPerThread; ++q) {
     const int64_t quad = quad0 + 32 * q;
     if (quad >= T.nquads) break;
-    const float4 vr = __ldcs(reinterpret_cast<const float4*>(T.w_re) + quad);
-    const float4 vi = __ldcs(reinterpret_cast<const float4*>(T.w_im) + quad);
-    const float wr[4] = {vr.x, vr.y, vr.z, vr.w};
-    const float wi[4] = {vi.x, vi.y, vi.z, vi.w};
-    uint32_t prev_bytes[IFQ_MAX_STAGES];
-    if (!FIRST) {
-#pragma unroll
-      for (int u = 0; u < IFQ_MAX_STAGES; ++u)
-        if (u < stage) prev_bytes[u] = __ldg(T.codes + (int64_t)u * T.nquads + quad);
-    }
-    uint32_t byte = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const bool finite = isfinite(wr[e]) && isfinite(wi[e]);
-      bad |= !finite;
-      uint32_t k;
-      if (FIRST) {
-        const float a = finite ? wr[e] : 0.0f;
-        const float b = finite ? wi[e] : 0.0f;
-        k = phase_sector(a, b);
-        if ((k & 1u) == 0u) {
-          S_re += (double)fabsf(a);
-          ++C_re;
-        } else {
-          S_im += (double)fabsf(b);
-        }
-      } else {
-        double a = finite ? (double)wr[e] : 0.0;
-        double b = finite ? (double)wi[e] : 0.0;
-#pragma unroll
-        for (int u = 0; u < IFQ_MAX_STAGES; ++u) {
-          if (u < stage) {
-            const uint32_t ku = (prev_bytes[u] >> (2 * e)) & 3u;
-            const double sgn = (ku & 2u) ? -1.0 : 1.0;
-            const double br = (ku & 1u) ? 0.0 : sgn;
-            const double bi = (ku & 1u) ? sgn : 0.0;
-            a = a - s_prev_re[u] * br;
-            b = b - s_prev_im[u] * bi;
-          }
-        }
-        k = phase_sector(a, b);
-        if ((k & 1u) == 0u) {
-          S_re += fabs(a);
-          ++C_re;
-        } else {
-          S_im += fabs(b);
-        }
-      }
-      byte |= k << (2 * e);
-    }
-    T.codes[(int64_t)stage * T.nquads + quad] = (uint8_t)byte;
+    const uint32_t byte = quad_code<PREV>(wr[q], wi[q], prev[q], sr, si, bad, S_re, S_im);
+    C_re += 4u - (uint32_t)__popc(byte & 0x55u);
+    T.codes[(int64_t)PREV * T.nquads + quad] = (uint8_t)byte;
   }
 
   if (__syncthreads_or(bad) && threadIdx.x == 0) set_status(p.status, IFQ_DEV_NONFINITE);
@@ -195,8 +215,8 @@ __global__ void __launch_bounds__(kQThreads) quant_stage_kernel(const __grid_con
     part.pad = 0;
     T.partials[blk] = part;
     __threadfence();
-    const unsigned prev = atomicAdd(T.ticket, 1u);
-    am_last = (prev == (unsigned)(T.nblocks - 1));
+    const unsigned prev_ticket = atomicAdd(T.ticket, 1u);
+    am_last = (prev_ticket == (unsigned)(T.nblocks - 1));
   }
   __syncthreads();
   if (!am_last) return;
@@ -217,10 +237,15 @@ __global__ void __launch_bounds__(kQThreads) quant_stage_kernel(const __grid_con
     const unsigned long long c_im = total - c;
     const float s_re = c > 0 ? (float)(a / (double)c) : 0.0f;
     const float s_im = c_im > 0 ? (float)(b / (double)c_im) : 0.0f;
-    T.scales[2 * stage] = s_re;
-    T.scales[2 * stage + 1] = s_im;
+    T.scales[2 * PREV] = s_re;
+    T.scales[2 * PREV + 1] = s_im;
     *T.ticket = 0u;  // re-arm for the next stage launch
   }
+}
+
+template <int PREV>
+void launch_stage(const QParams& p, unsigned blocks, cudaStream_t s) {
+  quant_stage_kernel<PREV><<<blocks, kQThreads, 0, s>>>(p);
 }
 
 }  // namespace
@@ -265,10 +290,17 @@ cudaError_t launch_quantize(const ifq_qtensor* t, int count, int T, void* ws, ui
   if (e != cudaSuccess) return e;
   for (int st = 0; st < T; ++st) {
     p.stage = st;
-    if (st == 0)
-      quant_stage_kernel<true><<<(unsigned)blocks, kQThreads, 0, s>>>(p);
-    else
-      quant_stage_kernel<false><<<(unsigned)blocks, kQThreads, 0, s>>>(p);
+    const unsigned nb = (unsigned)blocks;
+    switch (st) {
+      case 0: launch_stage<0>(p, nb, s); break;
+      case 1: launch_stage<1>(p, nb, s); break;
+      case 2: launch_stage<2>(p, nb, s); break;
+      case 3: launch_stage<3>(p, nb, s); break;
+      case 4: launch_stage<4>(p, nb, s); break;
+      case 5: launch_stage<5>(p, nb, s); break;
+      case 6: launch_stage<6>(p, nb, s); break;
+      default: launch_stage<7>(p, nb, s); break;
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

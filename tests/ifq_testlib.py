@@ -52,6 +52,15 @@ def gpu_quantize(ws, T, dev_status=None):
     return outs
 
 
+def run_gemv(descs, T, B, workspace=None, dev_status=None):
+    """Decode product through the C ABI; allocates a zero-filled workspace when none is given."""
+    if workspace is None:
+        n = Q.ifq_gemv_workspace_bytes(descs, T, B)
+        workspace = torch.zeros(max(n, 16), dtype=torch.uint8, device=DEV)
+    Q.ifq_gemv(descs, T, B, workspace=workspace, dev_status=dev_status)
+    return workspace
+
+
 def layer_desc(cu, su, cw, sw, x_re, x_im, N, K, rows):
     y_re = torch.empty((rows, N), dtype=torch.float32, device=DEV)
     y_im = torch.empty((rows, N), dtype=torch.float32, device=DEV)

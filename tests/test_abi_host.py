@@ -46,9 +46,9 @@ def _layer(**kw):
                    d["x_im"], d["y_re"], d["y_im"])
 
 
-def _call_gemv(layers, T=1, B=1):
+def _call_gemv(layers, T=1, B=1, ws=FAKE, ws_bytes=1 << 30):
     arr = (L.Layer * max(1, len(layers)))(*layers)
-    return Q.load().ifq_gemv(arr if layers else None, len(layers), T, B, None, None)
+    return Q.load().ifq_gemv(arr if layers else None, len(layers), T, B, ws, ws_bytes, None, None)
 
 
 def _call_gemm(layers, T=1, M=128):
@@ -77,7 +77,19 @@ def test_batch_stage_and_count_errors():
     assert _call_gemv([]) == 1
     many = [good] * 33
     arr = (L.Layer * 33)(*many)
-    assert Q.load().ifq_gemv(arr, 33, 1, 1, None, None) == 9
+    assert Q.load().ifq_gemv(arr, 33, 1, 1, FAKE, 1 << 30, None, None) == 9
+
+
+def test_gemv_workspace_errors():
+    good = _layer(N=300, K=5504)
+    lib = Q.load()
+    arr = (L.Layer * 1)(good)
+    need = lib.ifq_gemv_workspace_bytes(arr, 1, 2, 1)
+    assert need > 0
+    assert lib.ifq_gemv_workspace_bytes(arr, 1, 2, 4) == 0     # B >= 2 needs none
+    assert _call_gemv([good], T=2, B=1, ws=None, ws_bytes=need) == 6
+    assert _call_gemv([good], T=2, B=1, ws=FAKE, ws_bytes=need - 1) == 6
+    assert _call_gemv([good], T=2, B=1, ws=FAKE + 8, ws_bytes=need) == 3
 
 
 def test_quantize_argument_errors():

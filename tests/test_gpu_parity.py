@@ -9,7 +9,7 @@ import bit_complex_quantized_b200 as Q
 from bit_complex_quantized_b200 import workloads as W
 import oracle as O
 from ifq_testlib import (DEV, check_convert, check_product, check_quantized, gpu_convert, gpu_quantize,
-                         layer_desc, sample_rows, status_word, to_dev)
+                         layer_desc, run_gemv, sample_rows, status_word, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -45,7 +45,7 @@ def test_c1_single_layer_quantize_and_gemv():
     N, K = cfg.layers[0].N, cfg.layers[0].K
     xr, xi, xrn, xin = _x(cfg, 0, 1)
     d = layer_desc(codes, scales, None, None, xr, xi, N, K, 1)
-    Q.ifq_gemv([d], cfg.T, 1)
+    run_gemv([d], cfg.T, 1)
     torch.cuda.synchronize()
     check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cn, sn, None, None, xrn, xin)
 
@@ -65,7 +65,7 @@ def test_c2_block_quantize_gemv_b1_b8_and_gemm():
             xr, xi, xrn, xin = _x(cfg, i, B)
             xs.append((xrn, xin))
             descs.append(layer_desc(outs[i][0], outs[i][1], None, None, xr, xi, spec.N, spec.K, B))
-        Q.ifq_gemv(descs, cfg.T, B)
+        run_gemv(descs, cfg.T, B)
         torch.cuda.synchronize()
         for d, (cn, sn), (xrn, xin) in zip(descs, host, xs):
             check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cn, sn, None, None, xrn, xin)
@@ -125,7 +125,7 @@ def test_c3_gemv_b1_b16(c3_quantized):
             xs.append((xrn, xin))
             (cu, su), (cw, sw) = outs[2 * i], outs[2 * i + 1]
             descs.append(layer_desc(cu, su, cw, sw, xr, xi, spec.N, spec.K, B))
-        Q.ifq_gemv(descs, cfg.T, B)
+        run_gemv(descs, cfg.T, B)
         torch.cuda.synchronize()
         for i, (d, spec) in enumerate(zip(descs, cfg.layers)):
             (cun, sun), (cwn, swn) = host[2 * i], host[2 * i + 1]
@@ -163,7 +163,7 @@ def test_c3_gemv_and_gemm_agree_on_same_tokens(c3_quantized):
     (cu, su), (cw, sw) = outs[2 * i], outs[2 * i + 1]
     dv = layer_desc(cu, su, cw, sw, xr, xi, spec.N, spec.K, B)
     dm = layer_desc(cu, su, cw, sw, xr, xi, spec.N, spec.K, B)
-    Q.ifq_gemv([dv], cfg.T, B)
+    run_gemv([dv], cfg.T, B)
     Q.ifq_gemm([dm], cfg.T, B)
     torch.cuda.synchronize()
     bound = O.tolerance_bound(host[2 * i][1], host[2 * i + 1][1], xrn, xin)[:, None]
@@ -202,7 +202,7 @@ def test_c5_convert_quantize_gemv():
             xs.append((xrn, xin))
             (cu, su), (cw, sw) = outs_all[2 * i], outs_all[2 * i + 1]
             descs.append(layer_desc(cu, su, cw, sw, xr, xi, spec.N, spec.K, B))
-        Q.ifq_gemv(descs, cfg.T, B)
+        run_gemv(descs, cfg.T, B)
         torch.cuda.synchronize()
         for i, (d, spec) in enumerate(zip(descs, cfg.layers)):
             (cun, sun), (cwn, swn) = host_all[2 * i], host_all[2 * i + 1]
@@ -237,7 +237,7 @@ def test_ragged_shapes_all_batches(N, K, T, conj):
         xr = torch.from_numpy(xr32).to(torch.bfloat16)
         xi = torch.from_numpy(xi32).to(torch.bfloat16)
         d = layer_desc(cu, su, cw, sw, xr.to(DEV), xi.to(DEV), N, K, B)
-        Q.ifq_gemv([d], T, B)
+        run_gemv([d], T, B)
         torch.cuda.synchronize()
         check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cun, sun, cwn, swn,
                       W.bf16_to_f32_numpy(xr), W.bf16_to_f32_numpy(xi))
@@ -297,14 +297,20 @@ def test_gemv_and_quantizer_are_bit_reproducible():
     xi = torch.from_numpy(rng.standard_normal((4, K)).astype(np.float32)).to(torch.bfloat16).to(DEV)
     d1 = layer_desc(o1[0][0], o1[0][1], o1[1][0], o1[1][1], xr, xi, N, K, 4)
     d2 = layer_desc(o1[0][0], o1[0][1], o1[1][0], o1[1][1], xr, xi, N, K, 4)
-    Q.ifq_gemv([d1], T, 4)
-    Q.ifq_gemv([d2], T, 4)
+    run_gemv([d1], T, 4)
+    run_gemv([d2], T, 4)
+    # B = 1 integer path: two calls through one workspace (its tickets re-arm)
+    e1 = layer_desc(o1[0][0], o1[0][1], o1[1][0], o1[1][1], xr[:1].contiguous(), xi[:1].contiguous(), N, K, 1)
+    e2 = layer_desc(o1[0][0], o1[0][1], o1[1][0], o1[1][1], xr[:1].contiguous(), xi[:1].contiguous(), N, K, 1)
+    ws = run_gemv([e1], T, 1)
+    run_gemv([e2], T, 1, workspace=ws)
     m1 = layer_desc(o1[0][0], o1[0][1], o1[1][0], o1[1][1], xr, xi, N, K, 4)
     m2 = layer_desc(o1[0][0], o1[0][1], o1[1][0], o1[1][1], xr, xi, N, K, 4)
     Q.ifq_gemm([m1], T, 4)
     Q.ifq_gemm([m2], T, 4)
     torch.cuda.synchronize()
     assert torch.equal(d1["y_re"], d2["y_re"]) and torch.equal(d1["y_im"], d2["y_im"])
+    assert torch.equal(e1["y_re"], e2["y_re"]) and torch.equal(e1["y_im"], e2["y_im"])
     assert torch.equal(m1["y_re"], m2["y_re"]) and torch.equal(m1["y_im"], m2["y_im"])
 
 
@@ -316,3 +322,59 @@ def test_conversion_odd_width_and_subnormals():
     R2 = (0.02 * rng.standard_normal((64, 128))).astype(np.float32)
     R2[1, :4] = [1e-45, -1e-45, 2e-38, 0.0]
     check_convert(R2, gpu_convert(R2))
+
+
+# ---------------------------------------------------------------- B = 1 integer path
+def _b1_case(rng, N, K, T, conj, xr32, xi32):
+    ws = [_rand_complex(rng, N, K)] + ([_rand_complex(rng, N, K, 0.03)] if conj else [])
+    outs = gpu_quantize([(to_dev(a), to_dev(b)) for a, b in ws], T)
+    torch.cuda.synchronize()
+    host = [(c.cpu().numpy(), s.cpu().numpy()) for c, s in outs]
+    cu, su = outs[0]
+    cw, sw = outs[1] if conj else (None, None)
+    xr = torch.from_numpy(xr32).to(torch.bfloat16)
+    xi = torch.from_numpy(xi32).to(torch.bfloat16)
+    d = layer_desc(cu, su, cw, sw, xr.to(DEV), xi.to(DEV), N, K, 1)
+    st = status_word()
+    run_gemv([d], T, 1, dev_status=st)
+    torch.cuda.synchronize()
+    return d, host, W.bf16_to_f32_numpy(xr), W.bf16_to_f32_numpy(xi), int(st.item())
+
+
+@pytest.mark.parametrize("K", [64, 192, 1024, 1088, 2048, 5504])
+def test_b1_ragged_k_blocks(K):
+    rng = np.random.default_rng(K)
+    N, T = 77, 2
+    d, host, xr, xi, st = _b1_case(rng, N, K, T, True, rng.standard_normal((1, K)).astype(np.float32),
+                                   rng.standard_normal((1, K)).astype(np.float32))
+    assert st == 0
+    (cun, sun), (cwn, swn) = host
+    check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cun, sun, cwn, swn, xr, xi)
+
+
+def test_b1_activation_dynamic_range():
+    """One huge activation beside tiny and bf16-subnormal ones, an all-zero block, and an
+    imaginary plane of a different magnitude: the per-block power-of-two scaling keeps every
+    output inside the bound."""
+    rng = np.random.default_rng(31)
+    N, K, T = 64, 3072, 2
+    xr = (1e-30 * rng.standard_normal((1, K))).astype(np.float32)
+    xr[0, 5] = 3.0e4
+    xr[0, 1024:2048] = 0.0                      # an all-zero K block
+    xr[0, 2048:2060] = 3e-39                    # subnormal after bf16 rounding
+    xi = (1e-3 * rng.standard_normal((1, K))).astype(np.float32)
+    d, host, xrb, xib, st = _b1_case(rng, N, K, T, True, xr, xi)
+    assert st == 0
+    (cun, sun), (cwn, swn) = host
+    check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cun, sun, cwn, swn, xrb, xib)
+
+
+def test_b1_nonfinite_activation_is_flagged():
+    rng = np.random.default_rng(32)
+    N, K, T = 40, 128, 1
+    xr = rng.standard_normal((1, K)).astype(np.float32)
+    xi = rng.standard_normal((1, K)).astype(np.float32)
+    xr[0, 7] = np.inf
+    d, host, _, _, st = _b1_case(rng, N, K, T, False, xr, xi)
+    assert st & Q.IFQ_DEV_NONFINITE
+    assert torch.isnan(d["y_re"]).all()
