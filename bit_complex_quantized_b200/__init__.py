@@ -11,12 +11,14 @@ from ._lib import (  # noqa: F401
     IFQ_MAX_GEMV_BATCH,
     IFQ_MAX_GROUP,
     IFQ_MAX_STAGES,
+    IFQ_QUANT_STATIC_SCRATCH_BYTES,
     IfqError,
     LIB_PATH,
     ifq_gemm,
     ifq_gemv,
     ifq_gemv_workspace_bytes,
     ifq_quantize_pack,
+    ifq_quantize_pack_static,
     ifq_quantize_workspace_bytes,
     ifq_status_string,
     ifq_widely_linear_from_real,

@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(_PKG, "libifq.so")
 IFQ_MAX_STAGES = 8
 IFQ_MAX_GEMV_BATCH = 16
 IFQ_MAX_GROUP = 32
+IFQ_QUANT_STATIC_SCRATCH_BYTES = 2 << 20
 IFQ_DEV_NONFINITE = 0x1
 IFQ_DEV_TIMEOUT = 0x2
 
@@ -24,6 +25,7 @@ EXPORTED = (
     "ifq_widely_linear_from_real",
     "ifq_quantize_workspace_bytes",
     "ifq_quantize_pack",
+    "ifq_quantize_pack_static",
     "ifq_gemv_workspace_bytes",
     "ifq_gemv",
     "ifq_gemm",
@@ -32,6 +34,7 @@ EXPORTED = (
 STATUS_NAMES = {
     0: "IFQ_OK", 1: "IFQ_ERR_NULL", 2: "IFQ_ERR_SHAPE", 3: "IFQ_ERR_ALIGN", 4: "IFQ_ERR_STAGES",
     5: "IFQ_ERR_BATCH", 6: "IFQ_ERR_WORKSPACE", 7: "IFQ_ERR_CUDA", 8: "IFQ_ERR_UNSUPPORTED", 9: "IFQ_ERR_COUNT",
+    10: "IFQ_ERR_STATIC_LIMIT",
 }
 
 
@@ -73,6 +76,8 @@ def load():
     lib.ifq_quantize_workspace_bytes.argtypes = [ctypes.POINTER(QTensor), i32, i32]
     lib.ifq_quantize_pack.restype = i32
     lib.ifq_quantize_pack.argtypes = [ctypes.POINTER(QTensor), i32, i32, vp, sz, vp, vp]
+    lib.ifq_quantize_pack_static.restype = i32
+    lib.ifq_quantize_pack_static.argtypes = [ctypes.POINTER(QTensor), i32, i32, vp, vp]
     lib.ifq_gemv_workspace_bytes.restype = sz
     lib.ifq_gemv_workspace_bytes.argtypes = [ctypes.POINTER(Layer), i32, i32, i32]
     lib.ifq_gemv.restype = i32
@@ -129,6 +134,12 @@ def ifq_quantize_pack(tensors, T, workspace, dev_status=None, stream=None, works
     nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
     _check(load().ifq_quantize_pack(arr, len(tensors), T, _ptr(workspace), nbytes, _ptr(dev_status),
                                     _stream(stream)))
+
+
+def ifq_quantize_pack_static(tensors, T, dev_status=None, stream=None):
+    """As ifq_quantize_pack, with the library's fixed device scratch instead of a workspace."""
+    arr = _qtensors(tensors)
+    _check(load().ifq_quantize_pack_static(arr, len(tensors), T, _ptr(dev_status), _stream(stream)))
 
 
 def _layers(layers):

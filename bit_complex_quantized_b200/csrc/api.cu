@@ -58,6 +58,7 @@ const char* ifq_status_string(ifq_status s) {
     case IFQ_ERR_CUDA: return "CUDA runtime error";
     case IFQ_ERR_UNSUPPORTED: return "device is not sm_100";
     case IFQ_ERR_COUNT: return "descriptor count outside 1..32";
+    case IFQ_ERR_STATIC_LIMIT: return "call needs more than the 2 MiB static quantizer scratch";
   }
   return "unknown status";
 }
@@ -99,6 +100,25 @@ ifq_status ifq_quantize_pack(const ifq_qtensor* tensors, int count, int T, void*
   ifq_status st = check_device();
   if (st != IFQ_OK) return st;
   return from_cuda(ifq::launch_quantize(tensors, count, T, workspace, dev_status, as_stream(stream)));
+}
+
+ifq_status ifq_quantize_pack_static(const ifq_qtensor* tensors, int count, int T, uint32_t* dev_status,
+                                    ifq_stream_t stream) {
+  if (!tensors) return IFQ_ERR_NULL;
+  if (count < 1 || count > IFQ_MAX_GROUP) return IFQ_ERR_COUNT;
+  if (T < 1 || T > IFQ_MAX_STAGES) return IFQ_ERR_STAGES;
+  for (int i = 0; i < count; ++i) {
+    const ifq_qtensor& t = tensors[i];
+    if (!t.w_re || !t.w_im || !t.codes || !t.scales) return IFQ_ERR_NULL;
+    if (t.N < 1 || t.K < 4 || (t.K % 4) != 0) return IFQ_ERR_SHAPE;
+    if (t.K > (int64_t)1 << 30 || t.N > ((int64_t)1 << 40) / t.K) return IFQ_ERR_SHAPE;
+    if (!aligned16(t.w_re) || !aligned16(t.w_im) || !aligned16(t.codes) || (reinterpret_cast<uintptr_t>(t.scales) & 3u))
+      return IFQ_ERR_ALIGN;
+  }
+  if (ifq::quant_workspace_bytes(tensors, count) > IFQ_QUANT_STATIC_SCRATCH_BYTES) return IFQ_ERR_STATIC_LIMIT;
+  ifq_status st = check_device();
+  if (st != IFQ_OK) return st;
+  return from_cuda(ifq::launch_quantize_static(tensors, count, T, dev_status, as_stream(stream)));
 }
 
 size_t ifq_gemv_workspace_bytes(const ifq_layer* layers, int count, int T, int B) {

@@ -16,6 +16,8 @@ cudaError_t launch_widely_linear(const float* R, int64_t n, int64_t m, float* U_
 int64_t quant_blocks_for(int64_t N, int64_t K);
 size_t quant_workspace_bytes(const ifq_qtensor* t, int count);
 cudaError_t launch_quantize(const ifq_qtensor* t, int count, int T, void* ws, uint32_t* dev_status, cudaStream_t s);
+// As launch_quantize, with the scratch in a file-scope device array (no allocation).
+cudaError_t launch_quantize_static(const ifq_qtensor* t, int count, int T, uint32_t* dev_status, cudaStream_t s);
 
 cudaError_t launch_gemv(const ifq_layer* L, int count, int T, int B, uint32_t* dev_status, cudaStream_t s);
 

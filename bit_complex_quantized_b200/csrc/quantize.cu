@@ -20,6 +20,8 @@
 #include "ifq_common.cuh"
 #include "ifq_internal.h"
 
+#include <mutex>
+
 namespace ifq {
 namespace {
 
@@ -305,6 +307,32 @@ cudaError_t launch_quantize(const ifq_qtensor* t, int count, int T, void* ws, ui
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+// Scratch of ifq_quantize_pack_static, for callers that cannot hand over device
+// memory (a C loader without a device allocator, a server whose caches hold
+// the rest of the device).  Same layout as the caller workspace above.
+static __device__ __align__(256) unsigned char g_quant_scratch[IFQ_QUANT_STATIC_SCRATCH_BYTES];
+
+cudaError_t launch_quantize_static(const ifq_qtensor* t, int count, int T, uint32_t* dev_status, cudaStream_t s) {
+  constexpr int kCachedDevices = 64;
+  static std::mutex mu;
+  static void* addr[kCachedDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < kCachedDevices) scratch = addr[dev];
+    if (!scratch) {
+      // Once per device, with that device current: the array's address in its context.
+      e = cudaGetSymbolAddress(&scratch, g_quant_scratch);
+      if (e != cudaSuccess) return e;
+      if (dev >= 0 && dev < kCachedDevices) addr[dev] = scratch;
+    }
+  }
+  return launch_quantize(t, count, T, scratch, dev_status, s);
 }
 
 }  // namespace ifq

@@ -55,7 +55,8 @@ typedef enum {
   IFQ_ERR_WORKSPACE = 6,   /* workspace NULL or smaller than ifq_quantize_workspace_bytes() */
   IFQ_ERR_CUDA = 7,        /* a CUDA runtime call failed (launch error, no device, ...) */
   IFQ_ERR_UNSUPPORTED = 8, /* the device is not sm_100 */
-  IFQ_ERR_COUNT = 9        /* descriptor count outside 1..IFQ_MAX_GROUP */
+  IFQ_ERR_COUNT = 9,       /* descriptor count outside 1..IFQ_MAX_GROUP */
+  IFQ_ERR_STATIC_LIMIT = 10 /* the call needs more scratch than IFQ_QUANT_STATIC_SCRATCH_BYTES */
 } ifq_status;
 
 #define IFQ_MAX_STAGES 8
@@ -127,6 +128,38 @@ size_t ifq_quantize_workspace_bytes(const ifq_qtensor* tensors, int count, int T
 
 ifq_status ifq_quantize_pack(const ifq_qtensor* tensors, int count, int T, void* workspace,
                              size_t workspace_bytes, uint32_t* dev_status, ifq_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * ifq_quantize_pack_static
+ *
+ * The write-ups have no counterpart of this call: it is ifq_quantize_pack
+ * (same kernels, same results bit for bit) with its scratch in a fixed array
+ * inside the library instead of a caller workspace, for callers that cannot
+ * hand over device memory -- a plain C weight loader with no device allocator
+ * of its own, or a serving process that has reserved all free device memory
+ * for its caches before it quantizes.  Nothing is allocated: no cudaMalloc,
+ * no cudaFree, no allocating library call.
+ *
+ *   tensors, count, T, dev_status, stream   as for ifq_quantize_pack
+ *
+ * Limit: ifq_quantize_workspace_bytes(tensors, count, T) must not exceed
+ * IFQ_QUANT_STATIC_SCRATCH_BYTES (2 MiB: 32 bytes per 4096 complex weights,
+ * about 2.7e8 complex weights per call in total); larger calls return
+ * IFQ_ERR_STATIC_LIMIT before anything is launched.
+ * The part of the scratch that must start at zero (the per-tensor tickets) is
+ * cleared by every call with an asynchronous memset on `stream`.
+ * The first call on a device (with that device current) looks up the array's
+ * device address once (cudaGetSymbolAddress) and may load the library's device
+ * code; make that first call before anything that must not see such set-up,
+ * such as a stream capture.
+ * There is one array per device: calls whose work may overlap on the GPU
+ * (unordered streams, or several host threads) race on it and give wrong
+ * results.  Order such calls on one stream.
+ * ------------------------------------------------------------------------- */
+#define IFQ_QUANT_STATIC_SCRATCH_BYTES ((size_t)2 << 20)
+
+ifq_status ifq_quantize_pack_static(const ifq_qtensor* tensors, int count, int T, uint32_t* dev_status,
+                                    ifq_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Product layers ("Fairy2i write-up" §2.1, §4.2; "iFairy article" §二.2)
