@@ -80,8 +80,8 @@ struct I8Params {
 
 __device__ __forceinline__ void imma_16832(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                                            uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+  // Not volatile: a pure function of its registers, so the compiler may interleave it with loads.
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
@@ -92,12 +92,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
-}
-
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
 }
 
 __device__ __forceinline__ int find_layer_by(const I8Params& p, int64_t idx, bool prep) {
@@ -265,6 +259,30 @@ __device__ __forceinline__ int64_t warp_of_chunk(int64_t c, int64_t C, int64_t W
   return w;
 }
 
+// One chunk (16 rows x 256 positions) against this lane's 8 k-step fragments:
+// 16 MMAs, one per (in-byte position q, Gray plane), over the chunk's two word pairs.
+__device__ __forceinline__ void chunk_mma(int (&acc0)[4][4], int (&acc1)[4][4], const uint4* rowa, const uint4* rowb,
+                                          const uint4* fr) {
+  const uint4 va = *rowa, vb = *rowb;
+  uint4 F[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) F[k] = __ldg(fr + k);
+#pragma unroll
+  for (int wp = 0; wp < 2; ++wp) {
+    const uint32_t a0 = gray(wp ? va.z : va.x), a1 = gray(wp ? va.w : va.y);
+    const uint32_t b0 = gray(wp ? vb.z : vb.x), b1 = gray(wp ? vb.w : vb.y);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int ks = wp * 4 + q;
+      const uint32_t fx = (ks & 1) ? F[ks >> 1].z : F[ks >> 1].x;
+      const uint32_t fy = (ks & 1) ? F[ks >> 1].w : F[ks >> 1].y;
+      const uint32_t m0 = 0x01010101u << (2 * q), m1 = 0x02020202u << (2 * q);
+      imma_16832(acc0[q], a0 & m0, b0 & m0, a1 & m0, b1 & m0, fx, fy);
+      imma_16832(acc1[q], a0 & m1, b0 & m1, a1 & m1, b1 & m1, fx, fy);
+    }
+  }
+}
+
 // Lanes 0..15 each copy one code row of the piece into the slot.
 __device__ __forceinline__ void issue_piece(const I8Params& p, const Piece& pc, uint32_t slot, uint64_t* bar,
                                             int lane) {
@@ -289,6 +307,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3) gemv_i8_kernel(const __grid_co
   const int g = lane >> 2, tq = lane & 3;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * 2 * kSlotBytes) + warp * 2;
   const uint32_t slots = smem_u32(smem + warp * 2 * kSlotBytes);
+  const uint32_t slots0 = smem_u32(smem);
   if (lane == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
@@ -331,6 +350,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3) gemv_i8_kernel(const __grid_co
     int ok = 1;
     if (lane == 0) ok = mbar_wait_bounded_sleep(&bars[s], (phases >> s) & 1u, &abort_flag);
     ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();  // orders every lane's slot reads after lane 0's completed wait
     phases ^= 1u << s;
     if (!ok) {
       if (lane == 0) set_status(p.status, IFQ_DEV_TIMEOUT);
@@ -342,43 +362,21 @@ __global__ void __launch_bounds__(kWarps * 32, 3) gemv_i8_kernel(const __grid_co
     }
 
     const I8Layer& L = p.L[cur.li];
-    const uint32_t slot = slots + s * kSlotBytes;
+    const uint32_t slot = slots + s * kSlotBytes;  // shared-window address of this slot
     const int blk = cur.ch >> 3;
     // fragments of this piece's first chunk for this lane; 32 lanes x 64 B per chunk
     const uint4* fr = L.frag + (((int64_t)blk * 8 + (cur.ch & 7)) * 32 + lane) * 4;
-    const uint32_t rowa = slot + g * kSlotRow + tq * 16, rowb = rowa + 8 * kSlotRow;
+    // Plain shared loads (ordered after the barrier wait above by its memory clobber).
+    const uint4* rowa = reinterpret_cast<const uint4*>(smem + (slot - slots0) + g * kSlotRow + tq * 16);
+    const uint4* rowb = rowa + 8 * kSlotRow / 16;
 
     // Positions past K carry zero activation digits, so code bytes there (stale or not) add nothing.
-    // The next chunk's code words and fragments are loaded while this chunk computes.
-    uint4 va = lds128(rowa), vb = lds128(rowb);
-    uint4 F[4];
+    if (cur.len == kPieceChunks) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) F[k] = __ldg(fr + k);
-    for (int c = 0; c < cur.len; ++c) {
-      uint4 nva = va, nvb = vb, NF[4];
-      const int cn = c + 1 < cur.len ? c + 1 : c;
-      nva = lds128(rowa + cn * 64);
-      nvb = lds128(rowb + cn * 64);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) NF[k] = __ldg(fr + cn * 128 + k);
-#pragma unroll
-      for (int wp = 0; wp < 2; ++wp) {
-        const uint32_t a0 = gray(wp ? va.z : va.x), a1 = gray(wp ? va.w : va.y);
-        const uint32_t b0 = gray(wp ? vb.z : vb.x), b1 = gray(wp ? vb.w : vb.y);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int ks = wp * 4 + q;
-          const uint32_t fx = (ks & 1) ? F[ks >> 1].z : F[ks >> 1].x;
-          const uint32_t fy = (ks & 1) ? F[ks >> 1].w : F[ks >> 1].y;
-          const uint32_t m0 = 0x01010101u << (2 * q), m1 = 0x02020202u << (2 * q);
-          imma_16832(acc0[q], a0 & m0, b0 & m0, a1 & m0, b1 & m0, fx, fy);
-          imma_16832(acc1[q], a0 & m1, b0 & m1, a1 & m1, b1 & m1, fx, fy);
-        }
-      }
-      va = nva;
-      vb = nvb;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) F[k] = NF[k];
+      for (int c = 0; c < kPieceChunks; ++c) chunk_mma(acc0, acc1, rowa + c * 4, rowb + c * 4, fr + c * 128);
+    } else {
+#pragma unroll 1
+      for (int c = 0; c < cur.len; ++c) chunk_mma(acc0, acc1, rowa + c * 4, rowb + c * 4, fr + c * 128);
     }
     __syncwarp();  // every lane is done with this slot before it is refilled
 
