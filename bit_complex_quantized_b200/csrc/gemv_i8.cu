@@ -8,11 +8,12 @@
 //     Br = 1 - g0 - g1,   Bi = g0 - g1,
 // so two 0/1 bit-planes per code suffice:
 //     sum_j Br_j x_j = sum_j x_j - G0 - G1,   sum_j Bi_j x_j = G0 - G1,   G_b = sum_j g_b,j x_j.
-// In registers: gray = w ^ ((w >> 1) & 0x5555...), then one AND per (plane,
-// in-byte position q) selects 4 codes -- one per byte, all at position q -- as
-// int8 operands 4^q g0 or 2*4^q g1.  Each (plane, q) has its own int32
-// accumulator, so no shift is needed; the weights are undone exactly when the
-// accumulators are combined.
+// In registers both planes are read at bit 2q+1 of each byte (q: position of
+// the code in its byte): g1 = s is that bit of the code word w, g0 = c XOR s is
+// that bit of w ^ (w << 1).  One logic op per (plane, q) -- (w ^ 2w) & m or
+// w & m -- selects 4 codes, one per byte, as int8 operands 2*4^q g (-128 g at
+// q = 3).  Each (plane, q) has its own int32 accumulator, so no shift is
+// needed; the weights are undone exactly when the accumulators are combined.
 //
 // Activations.  ifq_gemv first runs gemv_prep_kernel: per block of up to 2048
 // K positions, x (bf16, both planes) is scaled by 2^E with the block maximum in
@@ -49,7 +50,9 @@ constexpr int kPieceChunks = 8;                // at most 8 chunks (256 K positi
 constexpr int kSlotRow = 576;                  // bytes per code row in a slot (512 + 64 pad: conflict-free)
 constexpr int kSlotBytes = 16 * kSlotRow;      // one 16-row slot
 constexpr int kMainSmem = kWarps * 2 * kSlotBytes + kWarps * 2 * 8;
-constexpr int kPrepThreads = 256;
+constexpr int kPrepThreads = 128;                // one item (plane, position, 16-group) per thread of a chunk
+constexpr int kCtasPerSm = 3;
+static_assert(kPieceChunks * 256 == kKBlock, "a piece is at most one K block, and one run of the int32 sums");
 
 struct I8Layer {
   const uint8_t* codes[2];
@@ -57,10 +60,11 @@ struct I8Layer {
   const uint16_t* x[2];
   float* y[2];
   uint4* frag;            // [blocks][8 chunks][32 lanes][4]: a lane's 8 k-step fragments of a chunk, contiguous
-  double* bsum;           // [blocks][2]
+  double* bsum;           // [blocks][9][2]: exact sums of v over the block's first c chunks, per plane
   int* bexp;              // [blocks]
   float* partials;        // [tiles][chunks per tile][16][2] (one slot per warp touching the tile)
-  unsigned int* tickets;  // [tiles]
+  int* next;              // [tiles][chunks per tile]: end of the portion that starts at this chunk
+  unsigned int* tickets;  // [tiles]: finished chunks of the tile
   int64_t N, K;
   int64_t chunk_begin;    // first global chunk
   int64_t prep_begin;     // first prep CTA
@@ -75,6 +79,7 @@ struct I8Params {
   int64_t total_chunks;
   int count;
   int T;
+  int sms;  // > 0: CTA b works as CTA (b % sms) * (gridDim / sms) + b / sms
   uint32_t* status;
 };
 
@@ -85,8 +90,6 @@ __device__ __forceinline__ void imma_16832(int (&c)[4], uint32_t a0, uint32_t a1
       : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-
-__device__ __forceinline__ uint32_t gray(uint32_t w) { return w ^ ((w >> 1) & 0x55555555u); }
 
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -101,8 +104,10 @@ __device__ __forceinline__ int find_layer_by(const I8Params& p, int64_t idx, boo
 }
 
 // ---------------------------------------------------------------- prep kernel
-// One CTA per (layer, K block): exponent, digit fragments, exact sums of v.
-// It also zeroes the layer's tile tickets for the main kernel.
+// One CTA per (layer, K block, 256-wide chunk): every CTA of a block finds the
+// block's exponent, then writes the digit fragments of its own chunk and the
+// exact sum of v up to its chunk's end (prefix sums at chunk boundaries).  The
+// first CTA of a layer also zeroes the layer's tile tickets.
 __global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(const __grid_constant__ I8Params p) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ __align__(16) uint16_t xs[2][kKBlock];
@@ -111,26 +116,31 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(const __grid_co
 
   const int li = find_layer_by(p, blockIdx.x, true);
   const I8Layer& L = p.L[li];
-  const int b = (int)(blockIdx.x - L.prep_begin);
+  const int bc = (int)(blockIdx.x - L.prep_begin);
+  const int b = bc >> 3, c = bc & 7;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (b == 0)
+  if (bc == 0)
     for (int t = tid; t < L.tiles; t += kPrepThreads) L.tickets[t] = 0u;
 
   const int64_t k0 = (int64_t)b * kKBlock;
   const int klen = (int)(L.K - k0 < kKBlock ? L.K - k0 : kKBlock);  // multiple of 64
-  const int nchunks = (klen + 255) >> 8;
+  if (c * 256 >= klen) return;  // the block's last chunk lies before this one
 
   unsigned int mx = 0;
-  for (int pl = 0; pl < 2; ++pl) {
-    const int idx = tid * 8;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (idx < klen) v = __ldg(reinterpret_cast<const uint4*>(L.x[pl] + k0 + idx));
-    *reinterpret_cast<uint4*>(&xs[pl][idx]) = v;
-    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      mx = max(mx, wv[q] & 0x7FFFu);
-      mx = max(mx, (wv[q] >> 16) & 0x7FFFu);
+  for (int r = 0; r < kKBlock / (8 * kPrepThreads); ++r) {
+#pragma unroll
+    for (int pl = 0; pl < 2; ++pl) {
+      const int idx = (r * kPrepThreads + tid) * 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (idx < klen) v = __ldg(reinterpret_cast<const uint4*>(L.x[pl] + k0 + idx));
+      *reinterpret_cast<uint4*>(&xs[pl][idx]) = v;
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        mx = max(mx, wv[q] & 0x7FFFu);
+        mx = max(mx, (wv[q] >> 16) & 0x7FFFu);
+      }
     }
   }
 #pragma unroll
@@ -147,17 +157,30 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(const __grid_co
     const int e = (f >> 23) ? (int)(f >> 23) - 127 : (31 - __clz(f)) - 149;
     E = 29 - e;
   }
-  if (nonfinite && tid == 0) set_status(p.status, IFQ_DEV_NONFINITE);
+  if (nonfinite && tid == 0 && c == 0) set_status(p.status, IFQ_DEV_NONFINITE);
   const int E1 = min(E, 127);
   const float f1 = __int_as_float((E1 + 127) << 23);
   const float f2 = __int_as_float((E - E1 + 127) << 23);
 
+  // Exact sum of v over positions [0, 256 (c + 1)) of the block, per plane (prefix sums
+  // at chunk boundaries): thread t adds positions t, t + 128, ... below the bound.
+  long long vsum = 0;
+  {
+    const int pl = tid & 1;
+    const int bound = (c + 1) * 256 < klen ? (c + 1) * 256 : klen;
+    for (int j = tid >> 1; j < bound; j += kPrepThreads / 2) {
+      if (!nonfinite) {
+        const float xf = __uint_as_float((uint32_t)xs[pl][j] << 16);
+        vsum += __float2int_rn((xf * f1) * f2);
+      }
+    }
+  }
   // Item (plane pl, in-byte position q, 16-position group grp = (chunk c, slice tq, word w))
   // covers positions grp*16 + 4i + q, i = 0..3: bytes i of the code word w at position q.
-  long long vsum = 0;
-  const int nitems = nchunks * 128;
-  for (int it = tid; it < nitems; it += kPrepThreads) {
-    const int pl = it & 1, q = (it >> 1) & 3, grp = it >> 3;
+  // One item per thread: the chunk's 128 items.
+  {
+    const int it = tid;
+    const int pl = it & 1, q = (it >> 1) & 3, grp = c * 16 + (it >> 3);
     uint32_t D[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -167,14 +190,13 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(const __grid_co
         const float xf = __uint_as_float((uint32_t)xs[pl][j] << 16);
         v = __float2int_rn((xf * f1) * f2);
       }
-      vsum += v;
       D[i] = ((uint32_t)v + 0x80808080u) ^ 0x80808080u;
     }
     const uint32_t lo01 = __byte_perm(D[0], D[1], 0x5140), lo23 = __byte_perm(D[2], D[3], 0x5140);
     const uint32_t hi01 = __byte_perm(D[0], D[1], 0x7362), hi23 = __byte_perm(D[2], D[3], 0x7362);
     const uint32_t dig[4] = {__byte_perm(lo01, lo23, 0x5410), __byte_perm(lo01, lo23, 0x7632),
                              __byte_perm(hi01, hi23, 0x5410), __byte_perm(hi01, hi23, 0x7632)};
-    const int c = grp >> 4, tqs = (grp >> 2) & 3, w = grp & 3;
+    const int tqs = (grp >> 2) & 3, w = grp & 3;
     const int ks = (w >> 1) * 4 + q;  // k-step within the chunk: (word pair, position)
     // a lane's fragments for chunk c: 8 k-steps x (b0, b1) = 64 contiguous bytes
     uint32_t* fr = reinterpret_cast<uint32_t*>(L.frag + ((int64_t)b * 8 + c) * 32 * 4) + ks * 2 + (w & 1);
@@ -189,8 +211,11 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(const __grid_co
     long long s = 0;
 #pragma unroll
     for (int w = 0; w < kPrepThreads / 32; ++w) s += ssum[tid][w];
-    L.bsum[2 * b + tid] = nonfinite ? __longlong_as_double(0x7FF8000000000000LL) : (double)s;
-    if (tid == 0) L.bexp[b] = E;
+    // prefix[c + 1]; the block's first CTA also writes prefix[0] = 0
+    double* pre = L.bsum + (int64_t)b * 18;
+    pre[(c + 1) * 2 + tid] = nonfinite ? __longlong_as_double(0x7FF8000000000000LL) : (double)s;
+    if (c == 0) pre[tid] = 0.0;
+    if (tid == 0 && c == 0) L.bexp[b] = E;
   }
 }
 
@@ -249,36 +274,53 @@ __device__ __forceinline__ Piece next_piece(const I8Params& p, const Piece& pc, 
   return n;
 }
 
-// Warp w < W owns chunks [lo(w), lo(w+1)) with lo(w) = floor(w C / W); W <= C.
+// Warp w < W owns chunks [lo(w), lo(w+1)) with lo(w) = floor(w C / W); W <= C, so no range is empty.
 __device__ __forceinline__ int64_t range_lo(int64_t w, int64_t C, int64_t W) { return (w * C) / W; }
 
-__device__ __forceinline__ int64_t warp_of_chunk(int64_t c, int64_t C, int64_t W) {
-  int64_t w = (c * W) / C;
-  while (w + 1 < W && range_lo(w + 1, C, W) <= c) ++w;
-  while (w > 0 && range_lo(w, C, W) > c) --w;
-  return w;
+
+// As imma_16832 with a zero accumulator input: starts a fresh sum without zeroing registers.
+__device__ __forceinline__ void imma_16832_first(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                 uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+      : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
+}
+
+__device__ __forceinline__ uint32_t xor_and(uint32_t a, uint32_t b, uint32_t c) {  // (a ^ b) & c in one op
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x28;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
 
 // One chunk (16 rows x 256 positions) against this lane's 8 k-step fragments:
 // 16 MMAs, one per (in-byte position q, Gray plane), over the chunk's two word pairs.
+// Both Gray planes are taken at bit 2q+1 of each byte: g1 = s is that bit of w,
+// and g0 = c XOR s is that bit of w ^ (w << 1), so no separate Gray step is needed.
+// kFirst: the piece's first chunk, whose first MMAs start the sums.
+template <bool kFirst>
 __device__ __forceinline__ void chunk_mma(int (&acc0)[4][4], int (&acc1)[4][4], const uint4* rowa, const uint4* rowb,
-                                          const uint4* fr) {
+                                          const uint4 (&F)[4]) {
   const uint4 va = *rowa, vb = *rowb;
-  uint4 F[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) F[k] = __ldg(fr + k);
 #pragma unroll
   for (int wp = 0; wp < 2; ++wp) {
-    const uint32_t a0 = gray(wp ? va.z : va.x), a1 = gray(wp ? va.w : va.y);
-    const uint32_t b0 = gray(wp ? vb.z : vb.x), b1 = gray(wp ? vb.w : vb.y);
+    const uint32_t a0 = wp ? va.z : va.x, a1 = wp ? va.w : va.y;
+    const uint32_t b0 = wp ? vb.z : vb.x, b1 = wp ? vb.w : vb.y;
+    const uint32_t a0s = a0 * 2u, a1s = a1 * 2u, b0s = b0 * 2u, b1s = b1 * 2u;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int ks = wp * 4 + q;
       const uint32_t fx = (ks & 1) ? F[ks >> 1].z : F[ks >> 1].x;
       const uint32_t fy = (ks & 1) ? F[ks >> 1].w : F[ks >> 1].y;
-      const uint32_t m0 = 0x01010101u << (2 * q), m1 = 0x02020202u << (2 * q);
-      imma_16832(acc0[q], a0 & m0, b0 & m0, a1 & m0, b1 & m0, fx, fy);
-      imma_16832(acc1[q], a0 & m1, b0 & m1, a1 & m1, b1 & m1, fx, fy);
+      const uint32_t m = 0x02020202u << (2 * q);
+      if (kFirst && wp == 0) {
+        imma_16832_first(acc0[q], xor_and(a0, a0s, m), xor_and(b0, b0s, m), xor_and(a1, a1s, m), xor_and(b1, b1s, m),
+                         fx, fy);
+        imma_16832_first(acc1[q], a0 & m, b0 & m, a1 & m, b1 & m, fx, fy);
+      } else {
+        imma_16832(acc0[q], xor_and(a0, a0s, m), xor_and(b0, b0s, m), xor_and(a1, a1s, m), xor_and(b1, b1s, m), fx,
+                   fy);
+        imma_16832(acc1[q], a0 & m, b0 & m, a1 & m, b1 & m, fx, fy);
+      }
     }
   }
 }
@@ -294,14 +336,14 @@ __device__ __forceinline__ void issue_piece(const I8Params& p, const Piece& pc, 
   if (lane == 0) mbar_arrive_expect_tx(bar, bytes * (uint32_t)rows);
   __syncwarp();
   if (lane < rows) {
-    const int t = pc.mat / L.nbranch, br = pc.mat % L.nbranch;
+    const int t = L.nbranch == 2 ? pc.mat >> 1 : pc.mat, br = L.nbranch == 2 ? pc.mat & 1 : 0;
     const int64_t rb = L.K >> 2;
     const uint8_t* src = L.codes[br] + ((int64_t)t * L.N + row0 + lane) * rb + (int64_t)pc.ch * 64;
     bulk_g2s(slot + lane * kSlotRow, src, bytes, bar);
   }
 }
 
-__global__ void __launch_bounds__(kWarps * 32, 3) gemv_i8_kernel(const __grid_constant__ I8Params p) {
+__global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_i8_kernel(const __grid_constant__ I8Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
@@ -319,7 +361,11 @@ __global__ void __launch_bounds__(kWarps * 32, 3) gemv_i8_kernel(const __grid_co
   // tile's chunks are consecutive.
   const int64_t C = p.total_chunks;
   const int64_t W = (int64_t)gridDim.x * kWarps < C ? (int64_t)gridDim.x * kWarps : C;
-  const int64_t gw = (int64_t)blockIdx.x * kWarps + warp;
+  // CTAs b, b + sms, ... usually share an SM; giving them adjacent ranges lets
+  // them share activation fragments in L1.
+  const int64_t lb = p.sms > 0 ? (int64_t)(blockIdx.x % p.sms) * (gridDim.x / p.sms) + blockIdx.x / p.sms
+                               : (int64_t)blockIdx.x;
+  const int64_t gw = lb * kWarps + warp;
   if (gw >= W) return;
   const int64_t c_lo = range_lo(gw, C, W), c_hi = range_lo(gw + 1, C, W);
 
@@ -332,12 +378,6 @@ __global__ void __launch_bounds__(kWarps * 32, 3) gemv_i8_kernel(const __grid_co
   issue_piece(p, cur, slots, &bars[0], lane);
   asm volatile("griddepcontrol.wait;" ::: "memory");
   double yr[2] = {0.0, 0.0}, yi[2] = {0.0, 0.0};  // rows g, g+8 of the current tile (tq == 0)
-  int acc0[4][4], acc1[4][4];  // [position q][fragment reg], summed over the pieces of one (tile, matrix, K block)
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-#pragma unroll
-    for (int r = 0; r < 4; ++r) acc0[q][r] = acc1[q][r] = 0;
-  bool first_of_block = (cur.ch & 7) == 0;  // this (tile, matrix, block) run starts the block
 
   for (;;) {
     const int64_t nc = cur.gbegin + cur.len;
@@ -347,6 +387,28 @@ __global__ void __launch_bounds__(kWarps * 32, 3) gemv_i8_kernel(const __grid_co
       nxt = next_piece(p, cur, c_hi);
       issue_piece(p, nxt, slots + (s ^ 1) * kSlotBytes, &bars[s ^ 1], lane);
     }
+    // While the codes are in flight: this lane's fragments of the piece's first
+    // chunk and the inputs of its combine step.
+    const I8Layer& L = p.L[cur.li];
+    const int blk = cur.ch >> 3;
+    const uint4* fr = L.frag + (((int64_t)blk * 8 + (cur.ch & 7)) * 32 + lane) * 4;  // 32 lanes x 64 B per chunk
+    uint4 F0[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) F0[k] = __ldg(fr + k);
+    const int t = L.nbranch == 2 ? cur.mat >> 1 : cur.mat, br = L.nbranch == 2 ? cur.mat & 1 : 0;
+    float sr = 0.0f, si = 0.0f;
+    int bexp = 0;
+    double bs_re = 0.0, bs_im = 0.0;
+    if (tq == 0) {
+      sr = __ldg(L.scales[br] + 2 * t);
+      si = __ldg(L.scales[br] + 2 * t + 1);
+      bexp = __ldg(L.bexp + blk);
+      // exact sums of v over the piece's chunks, from the prefix sums
+      const double* pre = L.bsum + (int64_t)blk * 18 + (cur.ch & 7) * 2;
+      bs_re = __ldg(pre + 2 * cur.len) - __ldg(pre);
+      bs_im = __ldg(pre + 2 * cur.len + 1) - __ldg(pre + 1);
+    }
+
     int ok = 1;
     if (lane == 0) ok = mbar_wait_bounded_sleep(&bars[s], (phases >> s) & 1u, &abort_flag);
     ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -361,101 +423,107 @@ __global__ void __launch_bounds__(kWarps * 32, 3) gemv_i8_kernel(const __grid_co
       return;
     }
 
-    const I8Layer& L = p.L[cur.li];
     const uint32_t slot = slots + s * kSlotBytes;  // shared-window address of this slot
-    const int blk = cur.ch >> 3;
-    // fragments of this piece's first chunk for this lane; 32 lanes x 64 B per chunk
-    const uint4* fr = L.frag + (((int64_t)blk * 8 + (cur.ch & 7)) * 32 + lane) * 4;
     // Plain shared loads (ordered after the barrier wait above by its memory clobber).
     const uint4* rowa = reinterpret_cast<const uint4*>(smem + (slot - slots0) + g * kSlotRow + tq * 16);
     const uint4* rowb = rowa + 8 * kSlotRow / 16;
 
+    int acc0[4][4], acc1[4][4];  // [position q][fragment reg]: the piece's int32 sums, started by chunk 0
     // Positions past K carry zero activation digits, so code bytes there (stale or not) add nothing.
     if (cur.len == kPieceChunks) {
+      uint4 Fc[4] = {F0[0], F0[1], F0[2], F0[3]};
 #pragma unroll
-      for (int c = 0; c < kPieceChunks; ++c) chunk_mma(acc0, acc1, rowa + c * 4, rowb + c * 4, fr + c * 128);
+      for (int c = 0; c < kPieceChunks; ++c) {
+        uint4 Fn[4];
+        if (c + 1 < kPieceChunks) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) Fn[k] = __ldg(fr + (c + 1) * 128 + k);
+        }
+        if (c == 0)
+          chunk_mma<true>(acc0, acc1, rowa, rowb, Fc);
+        else
+          chunk_mma<false>(acc0, acc1, rowa + c * 4, rowb + c * 4, Fc);
+        if (c + 1 < kPieceChunks) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) Fc[k] = Fn[k];
+        }
+      }
     } else {
+      chunk_mma<true>(acc0, acc1, rowa, rowb, F0);
 #pragma unroll 1
-      for (int c = 0; c < cur.len; ++c) chunk_mma(acc0, acc1, rowa + c * 4, rowb + c * 4, fr + c * 128);
+      for (int c = 1; c < cur.len; ++c) {
+        uint4 F[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) F[k] = __ldg(fr + c * 128 + k);
+        chunk_mma<false>(acc0, acc1, rowa + c * 4, rowb + c * 4, F);
+      }
     }
     __syncwarp();  // every lane is done with this slot before it is refilled
 
-    // The int32 sums stay open while the next piece continues the same (tile, matrix, K block).
-    const bool same_run = has_next && nxt.li == cur.li && nxt.tile == cur.tile && nxt.mat == cur.mat &&
-                          (nxt.ch >> 3) == blk;
-    if (!same_run) {
-    // ---- combine: weights 4^q (g0) and 2*4^q, -128 at q = 3 (g1) -> 64 G0 and 128 G1, exact int32
-    double qa[2], qb[2];  // rows g, g+8: this thread's two digit columns, combined
+    // ---- combine: both planes carry weights 2*4^q, -128 at q = 3 -> 128 G0 and 128 G1, exact int32.
+    // The digit columns are then merged in float32: its rounding (2^-24 of at most
+    // 3 sum_j |v_j| per piece) stays far inside the product tolerance.
+    float qa[2], qb[2];  // rows g, g+8: this thread's two digit columns, merged
     {
       int G0[4], G1[4];
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
-        G0[r] = 64 * acc0[0][r] + 16 * acc0[1][r] + 4 * acc0[2][r] + acc0[3][r];
+        G0[r] = 64 * acc0[0][r] + 16 * acc0[1][r] + 4 * acc0[2][r] - acc0[3][r];
         G1[r] = 64 * acc1[0][r] + 16 * acc1[1][r] + 4 * acc1[2][r] - acc1[3][r];
       }
-      const double dscale = (tq & 1) ? 65536.0 : 1.0;  // columns 2tq, 2tq+1 hold digits 2(tq&1), +1
-      qa[0] = dscale * ((double)G0[0] + 256.0 * (double)G0[1]);
-      qa[1] = dscale * ((double)G0[2] + 256.0 * (double)G0[3]);
-      qb[0] = dscale * ((double)G1[0] + 256.0 * (double)G1[1]);
-      qb[1] = dscale * ((double)G1[2] + 256.0 * (double)G1[3]);
+      const float dscale = (tq & 1) ? 65536.0f : 1.0f;  // columns 2tq, 2tq+1 hold digits 2(tq&1), +1
+      qa[0] = dscale * fmaf(256.0f, (float)G0[1], (float)G0[0]);
+      qa[1] = dscale * fmaf(256.0f, (float)G0[3], (float)G0[2]);
+      qb[0] = dscale * fmaf(256.0f, (float)G1[1], (float)G1[0]);
+      qb[1] = dscale * fmaf(256.0f, (float)G1[3], (float)G1[2]);
     }
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       qa[r] += __shfl_xor_sync(0xffffffffu, qa[r], 1);
       qb[r] += __shfl_xor_sync(0xffffffffu, qb[r], 1);
     }
-    double oa[2], ob[2];  // threads tq 0,1 hold plane re, 2,3 plane im: fetch the other plane
+    float oa[2], ob[2];  // threads tq 0,1 hold plane re, 2,3 plane im: fetch the other plane
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       oa[r] = __shfl_xor_sync(0xffffffffu, qa[r], 2);
       ob[r] = __shfl_xor_sync(0xffffffffu, qb[r], 2);
     }
     if (tq == 0) {
-      const int t = cur.mat / L.nbranch, br = cur.mat % L.nbranch;
-      const double sr = (double)__ldg(L.scales[br] + 2 * t), si = (double)__ldg(L.scales[br] + 2 * t + 1);
-      // the block sums of v count the whole block; a piece covers part of it, so use the
-      // sums only once per (tile, matrix, block): on the piece that starts the block's first chunk
-      const double inv = __longlong_as_double((long long)(1023 - L.bexp[blk]) << 52);  // 2^-E
+      const double inv = __longlong_as_double((long long)(1023 - bexp) << 52);  // 2^-E (outside float range)
+      const float fre = (float)bs_re, fim = (float)bs_im;
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
-        // G0 = QA / 64, G1 = QB / 128;  P_r = S - G0 - G1,  P_i = G0 - G1 (S added by the block's first piece)
-        const double Prr = -qa[r] * 0.015625 - qb[r] * 0.0078125;
-        const double Pir = qa[r] * 0.015625 - qb[r] * 0.0078125;
-        const double Pri = -oa[r] * 0.015625 - ob[r] * 0.0078125;
-        const double Pii = oa[r] * 0.015625 - ob[r] * 0.0078125;
-        double pr = 0.0, pi = 0.0;
-        if (first_of_block) {
-          pr = L.bsum[2 * blk];
-          pi = L.bsum[2 * blk + 1];
-        }
-        double vr, vi;
+        // G0 = QA / 128, G1 = QB / 128;  P_r = S - G0 - G1,  P_i = G0 - G1 (S: the piece's sums of v)
+        const float Prr = fre - (qa[r] + qb[r]) * 0.0078125f;
+        const float Pir = (qa[r] - qb[r]) * 0.0078125f;
+        const float Pri = fim - (oa[r] + ob[r]) * 0.0078125f;
+        const float Pii = (oa[r] - ob[r]) * 0.0078125f;
+        float vr, vi;
         if (br == 0) {
-          vr = sr * (Prr + pr) - si * Pii;
-          vi = sr * (Pri + pi) + si * Pir;
+          vr = sr * Prr - si * Pii;
+          vi = sr * Pri + si * Pir;
         } else {
-          vr = sr * (Prr + pr) + si * Pii;
-          vi = si * Pir - sr * (Pri + pi);
+          vr = sr * Prr + si * Pii;
+          vi = si * Pir - sr * Pri;
         }
-        yr[r] += vr * inv;
-        yi[r] += vi * inv;
+        yr[r] += (double)vr * inv;
+        yi[r] += (double)vi * inv;
       }
     }
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-#pragma unroll
-      for (int r = 0; r < 4; ++r) acc0[q][r] = acc1[q][r] = 0;
-    first_of_block = has_next && (nxt.ch & 7) == 0;
-    }  // !same_run
 
-    // ---- tile finished for this warp: write y, or a partial and possibly reduce
+    // ---- tile finished for this warp: write y, or a partial and possibly reduce.
+    // The tile's chunks [0, tc) are split into contiguous portions, one per warp
+    // that touched it.  A portion starting at local chunk c0 leaves its partial in
+    // slot c0 and the start of the next portion in next[c0]; the ticket counts
+    // finished chunks, and the warp that completes it adds the partials in chunk
+    // order, so the result does not depend on timing.
     const bool tile_done = !has_next || nxt.li != cur.li || nxt.tile != cur.tile;
     if (tile_done) {
       const int64_t tc = (int64_t)p.T * L.nbranch * L.nch;
       const int64_t tb = L.chunk_begin + cur.tile * tc;
-      const int64_t w_first = warp_of_chunk(tb, C, W), w_last = warp_of_chunk(tb + tc - 1, C, W);
-      const int nparts = (int)(w_last - w_first + 1);
+      const int64_t c0 = (c_lo > tb ? c_lo : tb) - tb, c1 = nc - tb;  // this warp's portion of the tile
       const int64_t row0 = cur.tile * 16;
-      if (nparts == 1) {
+      if (c0 == 0 && c1 == tc) {
         if (tq == 0) {
 #pragma unroll
           for (int r = 0; r < 2; ++r)
@@ -465,7 +533,8 @@ __global__ void __launch_bounds__(kWarps * 32, 3) gemv_i8_kernel(const __grid_co
             }
         }
       } else {
-        float* part = L.partials + (cur.tile * tc + (gw - w_first)) * 32;
+        const int64_t slot0 = cur.tile * tc;
+        float* part = L.partials + (slot0 + c0) * 32;
         if (tq == 0) {
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
@@ -473,19 +542,24 @@ __global__ void __launch_bounds__(kWarps * 32, 3) gemv_i8_kernel(const __grid_co
             part[2 * (g + 8 * r) + 1] = (float)yi[r];
           }
         }
+        if (lane == 0) L.next[slot0 + c0] = (int)c1;
         __threadfence();
         __syncwarp();
         unsigned prev = 0;
-        if (lane == 0) prev = atomicAdd(L.tickets + cur.tile, 1u);
+        if (lane == 0) prev = atomicAdd(L.tickets + cur.tile, (unsigned)(c1 - c0));
         prev = __shfl_sync(0xffffffffu, prev, 0);
-        if (prev == (unsigned)(nparts - 1)) {
+        if ((int64_t)prev + (c1 - c0) == tc) {
           __threadfence();
           if (lane < 16 && row0 + lane < L.N) {
-            const float* pt = L.partials + cur.tile * tc * 32 + 2 * lane;
             float ar = 0.0f, ai = 0.0f;
-            for (int k = 0; k < nparts; ++k) {
-              ar += __ldcg(pt + k * 32);
-              ai += __ldcg(pt + k * 32 + 1);
+            int64_t c = 0;
+            for (int64_t guard = 0; c < tc && guard < tc; ++guard) {
+              const float* pt = L.partials + (slot0 + c) * 32 + 2 * lane;
+              ar += __ldcg(pt);
+              ai += __ldcg(pt + 1);
+              const int64_t cn = __ldcg(L.next + slot0 + c);
+              if (cn <= c) break;  // cannot happen: portions are non-empty and ordered
+              c = cn;
             }
             L.y[0][row0 + lane] = ar;
             L.y[1][row0 + lane] = ai;
@@ -502,9 +576,10 @@ __global__ void __launch_bounds__(kWarps * 32, 3) gemv_i8_kernel(const __grid_co
 }
 
 // Workspace layout: 256 B header (unused), then per layer, each region
-// 256-byte aligned: fragments, block sums, block exponents, partials, tickets.
+// 256-byte aligned: fragments, chunk sums, block exponents, partials, portion
+// links, tickets.
 struct WsLayout {
-  size_t frag, bsum, bexp, part, tick;
+  size_t frag, bsum, bexp, part, next, tick;
 };
 
 inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -519,12 +594,14 @@ size_t layout_layers(const ifq_layer* Ls, int count, int T, WsLayout* out) {
     w.frag = off;
     off = align256(off + (size_t)blocks * 8 * 32 * 64);
     w.bsum = off;
-    off = align256(off + (size_t)blocks * 16);
+    off = align256(off + (size_t)blocks * 18 * 8);
     w.bexp = off;
     off = align256(off + (size_t)blocks * 4);
     const int64_t nch = (Ls[i].K + 255) / 256;
     w.part = off;
     off = align256(off + (size_t)tiles * nmat * nch * 32 * 4);
+    w.next = off;
+    off = align256(off + (size_t)tiles * nmat * nch * 4);
     w.tick = off;
     off = align256(off + (size_t)tiles * 4);
     if (out) out[i] = w;
@@ -571,12 +648,13 @@ cudaError_t launch_gemv_i8(const ifq_layer* Ls, int count, int T, void* ws, uint
     a.bsum = reinterpret_cast<double*>(base + lay[i].bsum);
     a.bexp = reinterpret_cast<int*>(base + lay[i].bexp);
     a.partials = reinterpret_cast<float*>(base + lay[i].part);
+    a.next = reinterpret_cast<int*>(base + lay[i].next);
     a.tickets = reinterpret_cast<unsigned int*>(base + lay[i].tick);
     a.nch = (int32_t)((a.K + 255) / 256);
     a.chunk_begin = chunks;
     a.prep_begin = preps;
     chunks += (int64_t)a.tiles * T * a.nbranch * a.nch;
-    preps += a.blocks;
+    preps += (int64_t)a.blocks * 8;
   }
   p.total_chunks = chunks;
   if (chunks >= ((int64_t)1 << 40) || preps > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
@@ -588,9 +666,10 @@ cudaError_t launch_gemv_i8(const ifq_layer* Ls, int count, int T, void* ws, uint
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int64_t ctas = (int64_t)sms * 3;
+  int64_t ctas = (int64_t)sms * kCtasPerSm;
   const int64_t need = (chunks + kWarps - 1) / kWarps;  // at least one chunk per warp
   if (ctas > need) ctas = need;
+  p.sms = ctas == (int64_t)sms * kCtasPerSm ? sms : 0;
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3((unsigned)ctas);
