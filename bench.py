@@ -292,6 +292,20 @@ def e2e_decode(block, steps, warmup):
             "d2h_bytes_per_step": d2h, "ms_per_step": t * 1e3}
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of every rank's values (times in seconds); a no-op on one rank."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def job_rate(world, units_per_rank, seconds):
+    """Whole-job throughput of `world` replicas that each processed `units_per_rank` in at most `seconds`."""
+    return world * units_per_rank / seconds
+
+
 # ---------------------------------------------------------------- main arm
 def run_ours(args):
     ws, rank, local = dist_env()
@@ -328,11 +342,8 @@ def run_ours(args):
     assert int(block.status.item()) == 0, "device status set during timing"
 
     # max over ranks of every time
-    vals = torch.tensor([total_s, per["convert"], per["quant"], per["gemv"], per["gemm"]], dtype=torch.float64,
-                        device=dev)
-    if ws > 1:
-        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
-    total_s, t_conv, t_quant, t_gemv, t_gemm = [float(v) for v in vals.cpu()]
+    total_s, t_conv, t_quant, t_gemv, t_gemm = max_over_ranks(
+        [total_s, per["convert"], per["quant"], per["gemv"], per["gemm"]], dev)
 
     pk, pk_src = peaks()
     hbm = float(pk["hbm_gbs"])
@@ -356,7 +367,7 @@ def run_ours(args):
     kernels = {
         "gemv": {"bound": "hbm", "achieved": gemv_gbs, "peak": hbm, "unit": "GB/s", "frac": gemv_gbs / hbm,
                  "us": t_gemv * 1e6, "algorithmic_bytes": gemv_bytes,
-                 "traffic": recorded_traffic("gemv.cu", "gemv", "c3_b1")},
+                 "traffic": recorded_traffic("gemv_i8.cu", "gemv", "c3_b1")},
         "gemm": {"bound": "tensor", "achieved": gemm_tops, "peak": tf_sus, "unit": "TFLOP/s",
                  "frac": gemm_tops / tf_sus, "us": t_gemm * 1e6, "equiv_flops": block.gemm_flops(),
                  "traffic": recorded_traffic("gemm.cu", "gemm", "c4_m2048")},
@@ -369,7 +380,7 @@ def run_ours(args):
     rl = dict(kernels[dominant])
     line = {
         "metric": METRIC,
-        "value": ws * gemv_gbs,
+        "value": job_rate(ws, gemv_bytes, t_gemv) / 1e9,
         "unit": "GB/s",
         "n_gpus": ws,
         "steps": args.steps,
@@ -384,7 +395,7 @@ def run_ours(args):
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
                    "l2": "256 MiB L2 flush before the GEMV in every step; conversion/quantizer inputs (1.6 GB) "
                          "exceed L2"},
-        "prefill_gemm": {"value": ws * gemm_tops, "unit": "TOP/s (equivalent dense, 8 M N K per stage and branch)",
+        "prefill_gemm": {"value": job_rate(ws, block.gemm_flops(), t_gemm) / 1e12, "unit": "TOP/s (equivalent dense, 8 M N K per stage and branch)",
                          "frac_of_sustained_bf16": gemm_tops / tf_sus},
         "roofline": {"kernel": dominant, "bound": rl["bound"], "achieved": rl["achieved"], "peak": rl["peak"],
                      "unit": rl["unit"], "frac": rl["frac"], "traffic": rl.get("traffic"),
@@ -431,9 +442,10 @@ def run_case(args):
     g = torch.Generator(device=dev)
     g.manual_seed(0)
     if args.case == "gemv":
-        # 70B-shaped layer set (321 MB of codes, larger than L2), random codes: the kernel's
-        # work does not depend on code values.
-        cfg = W.config("c5")
+        # 7B-shaped block (c3, 50.6 MB of codes) or 70B-shaped layer set (c5, 321 MB, larger
+        # than L2), random codes: the kernel's work does not depend on code values.  The L2 is
+        # flushed before every timed call.
+        cfg = W.config(args.workload)
         layers = []
         for i, spec in enumerate(cfg.layers):
             def rnd(shape):
@@ -451,7 +463,7 @@ def run_case(args):
 
         def fn():
             Q.ifq_gemv(layers, cfg.T, args.batch, workspace=gws)
-        label = f"gemv c5 B={args.batch}"
+        label = f"gemv {args.workload} B={args.batch}"
     elif args.case == "gemm":
         cfg = W.config("c4")
         spec = cfg.layers[4]  # gate: N = 5504, K = 2048
@@ -523,6 +535,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--case", choices=["gemv", "gemm", "quant", "convert"], default=None)
     ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--workload", choices=["c3", "c5"], default="c5", help="layer set of --case gemv")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     args = ap.parse_args()
