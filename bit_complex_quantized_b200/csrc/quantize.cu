@@ -119,22 +119,25 @@ __device__ __forceinline__ void block_sum3(double& a, double& b, unsigned long l
 // One quad (4 weights -> one code byte) of stage PREV (0-based), given the
 // earlier stages' code bytes of the quad.  Residual entries are rebuilt in
 // float64 one earlier stage at a time: Re r -= s_re Br, Im r -= s_im Bi, i.e.
-// add -s or +s when the code is on that axis.  Accumulates the quad's class
-// sums; returns the code byte.
+// add -s or +s when the code is on that axis.  The quad's four class values are
+// summed in float32 (at most 3 roundings of a sum of non-negative terms: below
+// 2e-7 relative) and that sum is added to the thread's float64 class sums.
+// Returns the code byte.
 template <int PREV>
 __device__ __forceinline__ uint32_t quad_code(const float (&wr)[4], const float (&wi)[4], const uint32_t (&prev)[8],
                                               const double (&sr)[8], const double (&si)[8], bool checked,
                                               double& S_re, double& S_im) {
   uint32_t byte = 0;
+  float q_re = 0.0f, q_im = 0.0f;
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     const bool fin = !checked || (isfinite(wr[e]) && isfinite(wi[e]));
     uint32_t k;
+    float v;
     if (PREV == 0) {
       const float a = fin ? wr[e] : 0.0f, b = fin ? wi[e] : 0.0f;
       k = sector_code(a, b);
-      const double v = (double)((k & 1u) ? fabsf(b) : fabsf(a));
-      if (k & 1u) S_im += v; else S_re += v;
+      v = (k & 1u) ? fabsf(b) : fabsf(a);
     } else {
       double a = fin ? (double)wr[e] : 0.0, b = fin ? (double)wi[e] : 0.0;
 #pragma unroll
@@ -146,11 +149,14 @@ __device__ __forceinline__ uint32_t quad_code(const float (&wr)[4], const float 
         b = (ku & 1u) ? b + step_i : b;
       }
       k = sector_code(a, b);
-      const double v = (k & 1u) ? fabs(b) : fabs(a);
-      if (k & 1u) S_im += v; else S_re += v;
+      v = (float)((k & 1u) ? fabs(b) : fabs(a));
     }
+    q_im += (k & 1u) ? v : 0.0f;
+    q_re += (k & 1u) ? 0.0f : v;
     byte |= k << (2 * e);
   }
+  S_re += (double)q_re;
+  S_im += (double)q_im;
   return byte;
 }
 
