@@ -168,8 +168,10 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(const __grid_co
   {
     const int pl = tid & 1;
     const int bound = (c + 1) * 256 < klen ? (c + 1) * 256 : klen;
-    for (int j = tid >> 1; j < bound; j += kPrepThreads / 2) {
-      if (!nonfinite) {
+#pragma unroll
+    for (int r = 0; r < kKBlock / (kPrepThreads / 2); ++r) {  // independent terms: unrolled for latency
+      const int j = (tid >> 1) + r * (kPrepThreads / 2);
+      if (j < bound && !nonfinite) {
         const float xf = __uint_as_float((uint32_t)xs[pl][j] << 16);
         vsum += __float2int_rn((xf * f1) * f2);
       }
@@ -274,6 +276,12 @@ __device__ __forceinline__ Piece next_piece(const I8Params& p, const Piece& pc, 
   return n;
 }
 
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* addr, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+  return old;
+}
+
 // Warp w < W owns chunks [lo(w), lo(w+1)) with lo(w) = floor(w C / W); W <= C, so no range is empty.
 __device__ __forceinline__ int64_t range_lo(int64_t w, int64_t C, int64_t W) { return (w * C) / W; }
 
@@ -372,11 +380,11 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_i8_kernel(const 
   int abort_flag = 0;
   uint32_t phases = 0u;  // bit s: parity of the next completion of slot s
   int s = 0;
-  // The code bytes do not depend on the prep kernel: start streaming them, then
-  // wait for the prep kernel's activation digits.
+  // The code bytes do not depend on the prep kernel: the first two pieces are
+  // put in flight before waiting for the prep kernel's activation digits.
   Piece cur = make_piece(p, c_lo, c_hi);
   issue_piece(p, cur, slots, &bars[0], lane);
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  bool prep_done = false;
   double yr[2] = {0.0, 0.0}, yi[2] = {0.0, 0.0};  // rows g, g+8 of the current tile (tq == 0)
 
   for (;;) {
@@ -386,6 +394,10 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_i8_kernel(const 
     if (has_next) {
       nxt = next_piece(p, cur, c_hi);
       issue_piece(p, nxt, slots + (s ^ 1) * kSlotBytes, &bars[s ^ 1], lane);
+    }
+    if (!prep_done) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      prep_done = true;
     }
     // While the codes are in flight: this lane's fragments of the piece's first
     // chunk and the inputs of its combine step.
@@ -543,13 +555,15 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_i8_kernel(const 
           }
         }
         if (lane == 0) L.next[slot0 + c0] = (int)c1;
-        __threadfence();
         __syncwarp();
         unsigned prev = 0;
-        if (lane == 0) prev = atomicAdd(L.tickets + cur.tile, (unsigned)(c1 - c0));
+        // acq_rel at gpu scope: the partial stores of the whole warp (ordered before
+        // lane 0 by the warp barrier above) are visible before the ticket moves, and
+        // the last arriver sees every other portion's stores after its own atomic.
+        if (lane == 0) prev = atom_add_acq_rel_gpu(L.tickets + cur.tile, (unsigned)(c1 - c0));
         prev = __shfl_sync(0xffffffffu, prev, 0);
         if ((int64_t)prev + (c1 - c0) == tc) {
-          __threadfence();
+          __syncwarp();
           if (lane < 16 && row0 + lane < L.N) {
             float ar = 0.0f, ai = 0.0f;
             int64_t c = 0;
