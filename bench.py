@@ -257,6 +257,42 @@ def oracle_decode_sample(seconds_budget=10.0, rows_per_layer=64, max_reps=50):
                       f"layers, U+W, T=2 ({nbytes / 1e6:.2f} MB of codes per rep), {reps} reps in {el:.1f} s"}
 
 
+# ---------------------------------------------------------------- dense comparator
+def dense_comparator(block, reps=20):
+    """Context, not the product: the original real layers of the block as dense bf16 matrices
+    multiplied by cuBLAS (torch.matmul) -- decode at B = 1 with an L2 flush before every call,
+    and prefill at the block's M.  Returns times and the ratios of our quantized path to them."""
+    dev = block.dev
+    Rs = [R.to(torch.bfloat16) for R in block.R]  # the block's real layers, already on the device
+    xs1 = [torch.randn((1, R.shape[1]), device=dev, dtype=torch.bfloat16) for R in Rs]
+    xsM = [torch.randn((block.M, R.shape[1]), device=dev, dtype=torch.bfloat16) for R in Rs]
+    weight_bytes = sum(R.numel() * 2 for R in Rs)
+
+    def timed(fn, flush):
+        times = []
+        for i in range(reps + 3):
+            if flush:
+                block.flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                times.append(a.elapsed_time(b) * 1e-3)
+        return statistics.median(times)
+
+    t_dec = timed(lambda: [torch.matmul(x, R.t()) for x, R in zip(xs1, Rs)], True)
+    t_pre = timed(lambda: [torch.matmul(x, R.t()) for x, R in zip(xsM, Rs)], False)
+    flops = sum(2 * block.M * R.shape[0] * R.shape[1] for R in Rs)
+    del Rs, xs1, xsM
+    return {"what": "cuBLAS bf16 matmul of the original real layers (7 layers, y = R x): decode B = 1 after an "
+                    "L2 flush, prefill M = %d" % block.M,
+            "decode_us": t_dec * 1e6, "decode_weight_bytes": weight_bytes,
+            "decode_GBps_of_weights": weight_bytes / t_dec / 1e9,
+            "prefill_us": t_pre * 1e6, "prefill_TFLOPs": flops / t_pre / 1e12}
+
+
 # ---------------------------------------------------------------- e2e
 def e2e_decode(block, steps, warmup):
     """Decode GEMV through the public API with host buffers: per step, pinned host -> device
@@ -359,6 +395,11 @@ def run_ours(args):
     cpu = None
     if rank == 0 and ws == 1 and not args.skip_cpu_baseline:
         cpu = oracle_decode_sample(seconds_budget=args.cpu_seconds)
+    dense = None
+    if rank == 0 and not args.skip_dense:
+        dense = dense_comparator(block)
+        dense["decode_ratio_quantized_to_dense_time"] = t_gemv / (dense["decode_us"] * 1e-6)
+        dense["prefill_ratio_quantized_to_dense_time"] = t_gemm / (dense["prefill_us"] * 1e-6)
     if ws > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -406,6 +447,7 @@ def run_ours(args):
         "kernels": kernels,
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "dense_bf16_comparator": dense,
         "gpu_launches": block.launches_per_step() * args.steps,
         "clocks": clk,
     }
@@ -538,6 +580,7 @@ def main():
     ap.add_argument("--workload", choices=["c3", "c5"], default="c5", help="layer set of --case gemv")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-dense", action="store_true", help="skip the cuBLAS bf16 dense comparator")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

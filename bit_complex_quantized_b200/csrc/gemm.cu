@@ -2,27 +2,34 @@
 // ("Fairy2i write-up" §2.1, §4.2; "iFairy article" §二.2 -- the GEMM rebuilt
 // from additions, subtractions and swaps).
 //
-// For each (stage t, branch) code matrix the per-class signed sums are one
-// real GEMM with exact operands:
-//     D_re = X_re [Br; Bi]^T,   D_im = X_im [Br; Bi]^T
-// X_* are the bf16 activation planes [M][K]; Br, Bi in {-2, 0, +2} are the
-// code's real / imaginary parts (times 2), expanded from the packed codes in
-// shared memory.  Products are exact and accumulate in float32 in TMEM, so the
-// +-1 and +-i classes keep separate accumulators (columns 0..63 and 64..127 of
-// each D) and their different scales are applied in the epilogue:
+// For each (stage t, branch) code matrix the per-class signed sums of one tile
+// are one real MMA with exact operands:
+//     D = [Br; Bi] [X_re; X_im]^T
+// Br, Bi in {-2, 0, +2} are the code's real / imaginary parts (times 2),
+// expanded from the packed codes straight into TMEM, where they are the MMA's
+// A operand (M = 128: Br and Bi rows of 64 outputs).  X_* are the bf16
+// activation planes [M][K], brought in by TMA; the two 128-token tiles of a K
+// block form the B operand (N = 256: real plane, then imaginary plane).
+// Products are exact and accumulate in float32 in TMEM; each lane holds one
+// (output, class) row and the columns hold (plane, token), so the four
+// quadrants are
+//     P_rr = Br x_re,  P_ri = Br x_im,  P_ir = Bi x_re,  P_ii = Bi x_im
+// and their scales are applied in the epilogue:
 //     U:  y_re += s_re P_rr - s_im P_ii,   y_im += s_re P_ri + s_im P_ir
 //     W:  y_re += s_re P_rr + s_im P_ii,   y_im += s_im P_ir - s_re P_ri
+// Keeping the expanded codes out of shared memory halves its traffic per MMA
+// (activations in by TMA and out to the tensor core, 16 KB per K16 step), so
+// the MMA is not starved by shared-memory bandwidth.
 //
-// CTA tile: 128 tokens (TMEM lanes) x 64 outputs; K in blocks of 64.
-// Warp roles (14 warps):
-//   0      TMA producer: X_re, X_im tiles (128 B swizzle) and the 64 x 16-byte code tile
-//   1      TMEM allocator and single-thread MMA issuer (M=128, N=128, K=16 per instruction)
-//   2-5    expanders: code tile -> B tile [Br rows 0..63; Bi rows 64..127] in the
-//          same 128 B-swizzled K-major layout the TMA uses for X
-//   6-13   epilogue: tcgen05.ld of the finished (stage, branch) accumulator,
-//          scale, accumulate y in registers; store y at the end
-// Accumulators are double-buffered (2 x 256 of the 512 TMEM columns) so the
-// epilogue of one (stage, branch) overlaps the main loop of the next.
+// CTA tile: 128 tokens x 64 outputs; K in blocks of 64.  Warp roles (10 warps):
+//   0-3   expanders: code tile -> A rows in TMEM (warp w writes lanes 32w..32w+31;
+//         lane 32w + j holds output 16w + (j & 15), class Br for j < 16, Bi else)
+//   4-7   epilogue: tcgen05.ld of the finished (stage, branch) accumulator, the
+//         Br/Bi exchange between lanes j and j ^ 16, scales, and y accumulated
+//         in shared memory; y stored to global at the end
+//   8     TMA producer: X_re, X_im tiles (128 B swizzle) and the 64 x 16-byte code tile
+//   9     TMEM allocator and single-thread MMA issuer (M=128, N=256, K=16 per instruction)
+// TMEM: the accumulator (256 columns) and 4 stages of A (32 columns each).
 // Every mbarrier wait is bounded; a lost wait sets IFQ_DEV_TIMEOUT, the CTA
 // drains its outstanding copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -35,19 +42,25 @@
 namespace ifq {
 namespace {
 
-constexpr int BM = 128;      // tokens per tile
-constexpr int BN = 64;       // outputs per tile
+constexpr int BM = 128;      // tokens per tile; the MMA's N is 2 BM (both planes)
+constexpr int BN = 64;       // outputs per tile; the MMA's M is 2 BN (Br and Bi rows)
 constexpr int BK = 64;       // K per stage (one 128-byte swizzle row of bf16)
 constexpr int STAGES = 4;
-constexpr int kThreads = 14 * 32;
+constexpr int kExpWarps = 4;
+constexpr int kEpiWarps = 4;
+constexpr int kProducerWarp = kExpWarps + kEpiWarps;
+constexpr int kMmaWarp = kProducerWarp + 1;
+constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr uint32_t kTileX = BM * BK * 2;        // 16 KB per activation plane
-constexpr uint32_t kTileB = 2 * BN * BK * 2;    // 16 KB: Br and Bi rows
 constexpr uint32_t kTileC = BN * (BK / 4);      // 1 KB of codes
-constexpr uint32_t kStageBytes = 2 * kTileX + kTileB + kTileC;  // 49 KB (multiple of 1 KB)
+constexpr uint32_t kStageBytes = 2 * kTileX + kTileC;  // 33 KB (multiple of 1 KB)
 constexpr uint32_t kTmaBytes = 2 * kTileX + kTileC;
-constexpr uint32_t kSmemBytes = STAGES * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+constexpr uint32_t kYFloats = 2 * BM * BN;      // y accumulators of the tile: [plane][token][output]
+constexpr uint32_t kSmemBytes = STAGES * kStageBytes + kYFloats * 4 + 1024 /*align*/ + 256 /*barriers*/;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kIdesc = umma_idesc_bf16(BM, 2 * BN);
+constexpr uint32_t kAcol = 2 * BM;              // A stage s at columns kAcol + 32 s
+constexpr uint32_t kIdesc = umma_idesc_bf16(2 * BN, 2 * BM);
+static_assert(kAcol + STAGES * (BK / 2) <= kTmemCols, "TMEM budget");
 
 struct __align__(64) GemmArgs {
   CUtensorMap tmap_x[2];      // bf16 [M][K]: box {64, 128}, 128 B swizzle
@@ -61,43 +74,29 @@ struct __align__(64) GemmArgs {
 
 struct Smem {
   uint64_t full_tma[STAGES];
-  uint64_t full_b[STAGES];
+  uint64_t full_a[STAGES];
   uint64_t empty[STAGES];
-  uint64_t acc_full[2];
-  uint64_t acc_empty[2];
+  uint64_t acc_full;
+  uint64_t acc_empty;
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
 
-// Source bits (from, from+1) of w moved to (to, to+1).
-__device__ __forceinline__ uint32_t move_bits(uint32_t w, int from, int to) {
-  return to >= from ? (w << (to - from)) : (w >> (from - to));
-}
-
-// Eight codes (j0..j0+7 of a 16-code word) -> 16 B of bf16 {Bi} and {Br} in K order.
-__device__ __forceinline__ void expand8(uint32_t w, int j0, uint4& bi, uint4& br) {
-  uint32_t o[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int j = j0 + 2 * q;
-    const uint32_t lo = move_bits(w, 2 * j, 14);      // code j   -> bits 14,15
-    const uint32_t hi = move_bits(w, 2 * j + 2, 30);  // code j+1 -> bits 30,31
-    o[q] = __byte_perm(lo, hi, 0x7610) & 0xC000C000u;
-  }
-  bi = make_uint4(o[0], o[1], o[2], o[3]);
-  br = make_uint4(o[0] ^ 0x40004000u, o[1] ^ 0x40004000u, o[2] ^ 0x40004000u, o[3] ^ 0x40004000u);
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
-  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
+// Two codes (bits 0..3 of `nib`) -> one 32-bit column of A: the bf16 pair (Br or Bi of the
+// lower code in the low half).  A code's axis bit lands on bit 14 (the exponent bit of 2.0)
+// and its sign bit on bit 15; the value is kept where the axis matches the class.
+__device__ __forceinline__ uint32_t expand_pair(uint32_t nib, bool imag) {
+  const uint32_t spread = ((nib & 3u) << 14) | ((nib >> 2) << 30);
+  const uint32_t u = imag ? spread : spread ^ 0x40004000u;  // bit 14 = "this code has the class's axis"
+  return u & ((u & 0x40004000u) * 3u);                      // keep exponent and sign only there
 }
 
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Smem* S = reinterpret_cast<Smem*>(smem + STAGES * kStageBytes);
+  float* ys = reinterpret_cast<float*>(smem + STAGES * kStageBytes);
+  Smem* S = reinterpret_cast<Smem*>(smem + STAGES * kStageBytes + kYFloats * 4);
   volatile int* abort = &S->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -106,21 +105,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   const int KB = (int)(a.K / BK);
   const int P = a.T * a.nbranch;
 
-  auto xre = [&](int s) { return smem + s * kStageBytes; };
-  auto xim = [&](int s) { return smem + s * kStageBytes + kTileX; };
-  auto btile = [&](int s) { return smem + s * kStageBytes + 2 * kTileX; };
-  auto ctile = [&](int s) { return smem + s * kStageBytes + 2 * kTileX + kTileB; };
+  auto xtile = [&](int s) { return smem + s * kStageBytes; };  // X_re, then X_im 16 KB later
+  auto ctile = [&](int s) { return smem + s * kStageBytes + 2 * kTileX; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&S->full_tma[s], 1);
-      mbar_init(&S->full_b[s], 4);
+      mbar_init(&S->full_a[s], kExpWarps);
       mbar_init(&S->empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&S->acc_full[b], 1);
-      mbar_init(&S->acc_empty[b], 8);
-    }
+    mbar_init(&S->acc_full, 1);
+    mbar_init(&S->acc_empty, kEpiWarps);
     mbar_init(&S->drain, 1);
     S->abort = 0;
     fence_mbar_init();
@@ -129,7 +124,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     prefetch_tmap(&a.tmap_codes[0]);
     if (a.nbranch > 1) prefetch_tmap(&a.tmap_codes[1]);
   }
-  if (warp == 1) {
+  for (uint32_t i = threadIdx.x; i < kYFloats; i += kThreads) ys[i] = 0.0f;
+  if (warp == kMmaWarp) {
     tmem_alloc(&S->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -138,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   tc_fence_after();
   const uint32_t tmem = S->tmem_base;
 
-  if (warp == 0) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int issued[STAGES];
@@ -151,8 +147,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
           if (!mbar_wait_bounded(&S->empty[s], ph ^ 1u, abort)) break;
           mbar_arrive_expect_tx(&S->full_tma[s], kTmaBytes);
-          tma_load_2d(xre(s), &a.tmap_x[0], kb * BK, (int32_t)m0, &S->full_tma[s]);
-          tma_load_2d(xim(s), &a.tmap_x[1], kb * BK, (int32_t)m0, &S->full_tma[s]);
+          tma_load_2d(xtile(s), &a.tmap_x[0], kb * BK, (int32_t)m0, &S->full_tma[s]);
+          tma_load_2d(xtile(s) + kTileX, &a.tmap_x[1], kb * BK, (int32_t)m0, &S->full_tma[s]);
           tma_load_2d(ctile(s), &a.tmap_codes[br], kb * (BK / 4), crow, &S->full_tma[s]);
           ++issued[s];
         }
@@ -164,34 +160,31 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           if (issued[s] > 0) mbar_wait_bounded(&S->full_tma[s], (uint32_t)(issued[s] - 1) & 1u, &never);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       for (int p = 0; p < P && !*abort; ++p) {
-        const int buf = p & 1;
-        if (!mbar_wait_bounded(&S->acc_empty[buf], ((uint32_t)(p >> 1) & 1u) ^ 1u, abort)) break;
+        // the epilogue has read the previous (stage, branch) accumulator
+        if (!mbar_wait_bounded(&S->acc_empty, ((uint32_t)p & 1u) ^ 1u, abort)) break;
         tc_fence_after();
-        const uint32_t d_re = tmem + buf * 256, d_im = d_re + 128;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
           const int it = p * KB + kb, s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!mbar_wait_bounded(&S->full_tma[s], ph, abort) || !mbar_wait_bounded(&S->full_b[s], ph, abort)) {
+          if (!mbar_wait_bounded(&S->full_tma[s], ph, abort) || !mbar_wait_bounded(&S->full_a[s], ph, abort)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t ar = smem_u32(xre(s)), ai = smem_u32(xim(s)), bb = smem_u32(btile(s));
+          const uint32_t xb = smem_u32(xtile(s));
 #pragma unroll
-          for (int ks = 0; ks < BK / 16; ++ks) {
-            const uint32_t acc = (kb | ks) != 0;
-            umma_bf16(d_re, umma_desc_sw128(ar + ks * 32), umma_desc_sw128(bb + ks * 32), kIdesc, acc);
-            umma_bf16(d_im, umma_desc_sw128(ai + ks * 32), umma_desc_sw128(bb + ks * 32), kIdesc, acc);
-          }
+          for (int ks = 0; ks < BK / 16; ++ks)
+            umma_bf16_ta(tmem, tmem + kAcol + 32 * s + 8 * ks, umma_desc_sw128(xb + ks * 32), kIdesc,
+                         (kb | ks) != 0);
           umma_commit(&S->empty[s]);
         }
         if (!ok) break;
-        umma_commit(&S->acc_full[buf]);
+        umma_commit(&S->acc_full);
       }
       if (*abort) {
         volatile int never = 0;
@@ -199,11 +192,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         mbar_wait_bounded(&S->drain, 0u, &never);
       }
     }
-  } else if (warp < 6) {
+  } else if (warp < kExpWarps) {
     // ------------------------------------------------------------ expanders
-    const int e = threadIdx.x - 64;  // 0..127
-    const int r = e >> 1, hf = e & 1;
-    const bool row_ok = n0 + r < a.N;
+    const bool imag = lane >= 16;
+    const int o = 16 * warp + (lane & 15);   // this lane's output row within the tile
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16) + kAcol;
     for (int p = 0; p < P && !__shfl_sync(0xffffffffu, *abort, 0); ++p) {
       for (int kb = 0; kb < KB; ++kb) {
         const int it = p * KB + kb, s = it % STAGES;
@@ -212,82 +205,81 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         if (lane == 0)
           ok = mbar_wait_bounded(&S->empty[s], ph ^ 1u, abort) && mbar_wait_bounded(&S->full_tma[s], ph, abort);
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-        const uint2 cw = row_ok ? *reinterpret_cast<const uint2*>(ctile(s) + r * 16 + hf * 8) : make_uint2(0, 0);
-        const uint32_t brow = smem_u32(btile(s)) + r * 128;
-        const uint32_t birow = brow + BN * 128;
+        // Rows past N carry other stages' or no codes; their outputs are never stored.
+        const uint4 cw = *reinterpret_cast<const uint4*>(ctile(s) + o * 16);
+        const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+        uint32_t col[32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint4 bi, brr;
-          expand8(c < 2 ? cw.x : cw.y, (c & 1) * 8, bi, brr);
-          if (!row_ok) bi = brr = make_uint4(0, 0, 0, 0);
-          const int chunk = hf * 4 + c;
-          const uint32_t off = (uint32_t)((chunk ^ (r & 7)) * 16);
-          st_shared_v4(brow + off, brr);
-          st_shared_v4(birow + off, bi);
-        }
-        fence_proxy_async_smem();
+        for (int c = 0; c < 32; ++c) col[c] = expand_pair((w[c >> 3] >> (4 * (c & 7))) & 0xFu, imag);
+        tmem_st_32x32b_x32(trow + 32 * s, col);
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S->full_b[s]);
+        if (lane == 0) mbar_arrive(&S->full_a[s]);
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int e = warp - 6;             // 0..7
-    const int q = warp & 3;             // TMEM lane quarter this warp may access
-    const int hc = e >> 2;              // output half: columns 32*hc .. 32*hc+31
-    float yr[32], yi[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) yr[j] = yi[j] = 0.0f;
+    const int q = warp - kExpWarps;          // TMEM lane quarter
+    const bool imag = lane >= 16;
+    const int o = 16 * q + (lane & 15);
+    const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
     for (int p = 0; p < P && !__shfl_sync(0xffffffffu, *abort, 0); ++p) {
-      const int buf = p & 1;
       int ok = 1;
-      if (lane == 0) ok = mbar_wait_bounded(&S->acc_full[buf], (uint32_t)(p >> 1) & 1u, abort);
+      if (lane == 0) ok = mbar_wait_bounded(&S->acc_full, (uint32_t)p & 1u, abort);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       tc_fence_after();
       const int t = p / a.nbranch, br = p % a.nbranch;
       const float hr = 0.5f * __ldg(a.scales[br] + 2 * t);
       const float hi = 0.5f * __ldg(a.scales[br] + 2 * t + 1);
-      const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + buf * 256 + hc * 32;
       const float sgn = br == 0 ? -1.0f : 1.0f;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t u[16], v[16];
-        tmem_ld_32x32b_x16(base + h * 16, u);             // P_rr
-        tmem_ld_32x32b_x16(base + 128 + 64 + h * 16, v);  // P_ii
+#pragma unroll 1
+      for (int c = 0; c < BM / 32; ++c) {
+        uint32_t u[32], v[32];
+        tmem_ld_32x32b_x32(trow + 32 * c, u);         // this lane's class, real plane, tokens 32c..
+        tmem_ld_32x32b_x32(trow + BM + 32 * c, v);    // imaginary plane
         tmem_wait_ld();
+        // lane j < 16 (Br) takes tokens 32c + 0..15, lane j >= 16 (Bi) tokens 32c + 16..31;
+        // each gets the other class's values of its tokens from lane j ^ 16
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          yr[h * 16 + j] += hr * __uint_as_float(u[j]) + sgn * hi * __uint_as_float(v[j]);
-        tmem_ld_32x32b_x16(base + 128 + h * 16, u);       // P_ri
-        tmem_ld_32x32b_x16(base + 64 + h * 16, v);        // P_ir
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          yi[h * 16 + j] += hi * __uint_as_float(v[j]) - sgn * hr * __uint_as_float(u[j]);
+        for (int i = 0; i < 16; ++i) {
+          const float mu_lo = __uint_as_float(u[i]), mv_lo = __uint_as_float(v[i]);
+          const float mu_hi = __uint_as_float(u[16 + i]), mv_hi = __uint_as_float(v[16 + i]);
+          // send the partner the values of the partner's tokens, receive those of mine
+          const float pu = __shfl_xor_sync(0xffffffffu, imag ? mu_lo : mu_hi, 16);
+          const float pv = __shfl_xor_sync(0xffffffffu, imag ? mv_lo : mv_hi, 16);
+          const float mu = imag ? mu_hi : mu_lo, mv = imag ? mv_hi : mv_lo;
+          const float P_rr = imag ? pu : mu, P_ri = imag ? pv : mv;
+          const float P_ir = imag ? mu : pu, P_ii = imag ? mv : pv;
+          const int tok = 32 * c + (imag ? 16 : 0) + i;
+          float* yre = ys + tok * BN + o;
+          float* yim = ys + BM * BN + tok * BN + o;
+          *yre += hr * P_rr + sgn * hi * P_ii;
+          *yim += hi * P_ir - sgn * hr * P_ri;
+        }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&S->acc_empty[buf]);
+      if (lane == 0) mbar_arrive(&S->acc_empty);
     }
+    // all epilogue warps have finished the tile's y: store it (rows of 64 outputs, float4)
+    asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
     if (!__shfl_sync(0xffffffffu, *abort, 0)) {
-      const int64_t m = m0 + q * 32 + lane;
-      const int64_t nb = n0 + hc * 32;
-      if (m < a.M) {
-        float* yre = a.y[0] + m * a.N + nb;
-        float* yim = a.y[1] + m * a.N + nb;
-        if ((a.N & 3) == 0 && nb + 32 <= a.N) {
-#pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            *reinterpret_cast<float4*>(yre + j) = make_float4(yr[j], yr[j + 1], yr[j + 2], yr[j + 3]);
-            *reinterpret_cast<float4*>(yim + j) = make_float4(yi[j], yi[j + 1], yi[j + 2], yi[j + 3]);
-          }
+      const int e = threadIdx.x - kExpWarps * 32;  // 0..127
+      const bool vec = (a.N & 3) == 0 && n0 + BN <= a.N;
+      for (int idx = e; idx < 2 * BM * (BN / 4); idx += kEpiWarps * 32) {
+        const int pl = idx / (BM * (BN / 4)), rem = idx - pl * (BM * (BN / 4));
+        const int tok = rem / (BN / 4), c4 = rem - tok * (BN / 4);
+        const int64_t m = m0 + tok;
+        if (m >= a.M) continue;
+        const float4 v4 = *reinterpret_cast<const float4*>(ys + pl * BM * BN + tok * BN + 4 * c4);
+        float* dst = a.y[pl] + m * a.N + n0 + 4 * c4;
+        if (vec) {
+          *reinterpret_cast<float4*>(dst) = v4;
         } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (nb + j < a.N) {
-              yre[j] = yr[j];
-              yim[j] = yi[j];
-            }
+          const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+          for (int j = 0; j < 4; ++j)
+            if (n0 + 4 * c4 + j < a.N) dst[j] = vv[j];
         }
       }
     }
@@ -296,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && S->abort) set_status(a.status, IFQ_DEV_TIMEOUT);
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }

@@ -378,3 +378,41 @@ def test_b1_nonfinite_activation_is_flagged():
     d, host, _, _, st = _b1_case(rng, N, K, T, False, xr, xi)
     assert st & Q.IFQ_DEV_NONFINITE
     assert torch.isnan(d["y_re"]).all()
+
+
+def test_max_group_of_32_layers():
+    """IFQ_MAX_GROUP layers in one grouped call: mixed shapes, every fourth layer with the conj
+    branch, at B = 1 (integer path: layer changes inside warp ranges) and B = 5 (bf16 path)."""
+    rng = np.random.default_rng(3232)
+    T = 2
+    specs = [(16 + 8 * (i % 9), (64, 128, 256, 320, 2112)[i % 5], i % 4 == 0) for i in range(Q.IFQ_MAX_GROUP)]
+    weights = []
+    for N, K, conj in specs:
+        weights.append([_rand_complex(rng, N, K)] + ([_rand_complex(rng, N, K, 0.03)] if conj else []))
+    flat = [w for ws in weights for w in ws]
+    outs = []
+    for i in range(0, len(flat), Q.IFQ_MAX_GROUP):  # quantizer groups of at most 32 tensors
+        outs += gpu_quantize([(to_dev(a), to_dev(b)) for a, b in flat[i:i + Q.IFQ_MAX_GROUP]], T)
+    torch.cuda.synchronize()
+    host = [(c.cpu().numpy(), s.cpu().numpy()) for c, s in outs]
+    for (wr, wi), (cn, sn) in zip(flat, host):
+        check_quantized(wr, wi, cn, sn, T)
+    for B in (1, 5):
+        descs, ref = [], []
+        j = 0
+        for (N, K, conj) in specs:
+            cu, su = outs[j]
+            cun, sun = host[j]
+            cw, sw, cwn, swn = (outs[j + 1][0], outs[j + 1][1], host[j + 1][0], host[j + 1][1]) if conj else \
+                (None, None, None, None)
+            j += 2 if conj else 1
+            xr = torch.from_numpy(rng.standard_normal((B, K)).astype(np.float32)).to(torch.bfloat16)
+            xi = torch.from_numpy(rng.standard_normal((B, K)).astype(np.float32)).to(torch.bfloat16)
+            descs.append(layer_desc(cu, su, cw, sw, xr.to(DEV), xi.to(DEV), N, K, B))
+            ref.append((cun, sun, cwn, swn, W.bf16_to_f32_numpy(xr), W.bf16_to_f32_numpy(xi)))
+        st = status_word()
+        run_gemv(descs, T, B, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        for d, (cun, sun, cwn, swn, xrn, xin) in zip(descs, ref):
+            check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cun, sun, cwn, swn, xrn, xin)
