@@ -21,14 +21,14 @@
 // (activations in by TMA and out to the tensor core, 16 KB per K16 step), so
 // the MMA is not starved by shared-memory bandwidth.
 //
-// CTA tile: 128 tokens x 64 outputs; K in blocks of 64.  Warp roles (10 warps):
+// CTA tile: 128 tokens x 64 outputs; K in blocks of 64.  Warp roles (14 warps):
 //   0-3   expanders: code tile -> A rows in TMEM (warp w writes lanes 32w..32w+31;
 //         lane 32w + j holds output 16w + (j & 15), class Br for j < 16, Bi else)
-//   4-7   epilogue: tcgen05.ld of the finished (stage, branch) accumulator, the
+//   4-11  epilogue: tcgen05.ld of the finished (stage, branch) accumulator, the
 //         Br/Bi exchange between lanes j and j ^ 16, scales, and y accumulated
 //         in shared memory; y stored to global at the end
-//   8     TMA producer: X_re, X_im tiles (128 B swizzle) and the 64 x 16-byte code tile
-//   9     TMEM allocator and single-thread MMA issuer (M=128, N=256, K=16 per instruction)
+//   12    TMA producer: X_re, X_im tiles (128 B swizzle) and the 64 x 16-byte code tile
+//   13    TMEM allocator and single-thread MMA issuer (M=128, N=256, K=16 per instruction)
 // TMEM: the accumulator (256 columns) and 4 stages of A (32 columns each).
 // Every mbarrier wait is bounded; a lost wait sets IFQ_DEV_TIMEOUT, the CTA
 // drains its outstanding copies and MMAs, frees TMEM and returns.
@@ -47,7 +47,7 @@ constexpr int BN = 64;       // outputs per tile; the MMA's M is 2 BN (Br and Bi
 constexpr int BK = 64;       // K per stage (one 128-byte swizzle row of bf16)
 constexpr int STAGES = 4;
 constexpr int kExpWarps = 4;
-constexpr int kEpiWarps = 4;
+constexpr int kEpiWarps = 8;                 // two per TMEM lane quarter, each half the tokens
 constexpr int kProducerWarp = kExpWarps + kEpiWarps;
 constexpr int kMmaWarp = kProducerWarp + 1;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
@@ -84,12 +84,13 @@ struct Smem {
 };
 
 // Two codes (bits 0..3 of `nib`) -> one 32-bit column of A: the bf16 pair (Br or Bi of the
-// lower code in the low half).  A code's axis bit lands on bit 14 (the exponent bit of 2.0)
-// and its sign bit on bit 15; the value is kept where the axis matches the class.
+// lower code in the low half).  The multiply places code 0's axis bit on bit 14 (the exponent
+// bit of 2.0) and its sign on bit 15, code 1's on bits 30 and 31.  Bi is then +-2 where the
+// axis bit is set and +-0 where it is not; Br flips the axis bit.  A signed zero adds nothing
+// to the float32 sums, so no further masking is needed.
 __device__ __forceinline__ uint32_t expand_pair(uint32_t nib, bool imag) {
-  const uint32_t spread = ((nib & 3u) << 14) | ((nib >> 2) << 30);
-  const uint32_t u = imag ? spread : spread ^ 0x40004000u;  // bit 14 = "this code has the class's axis"
-  return u & ((u & 0x40004000u) * 3u);                      // keep exponent and sign only there
+  const uint32_t spread = (nib * 0x10004000u) & 0xC000C000u;
+  return imag ? spread : spread ^ 0x40004000u;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ GemmArgs a) {
@@ -220,7 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp - kExpWarps;          // TMEM lane quarter
+    const int q = warp & 3;                  // TMEM lane quarter
+    const int half = (warp - kExpWarps) >> 2;  // token chunks c with c % 2 == half
     const bool imag = lane >= 16;
     const int o = 16 * q + (lane & 15);
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
@@ -234,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       const float hi = 0.5f * __ldg(a.scales[br] + 2 * t + 1);
       const float sgn = br == 0 ? -1.0f : 1.0f;
 #pragma unroll 1
-      for (int c = 0; c < BM / 32; ++c) {
+      for (int c = half; c < BM / 32; c += 2) {
         uint32_t u[32], v[32];
         tmem_ld_32x32b_x32(trow + 32 * c, u);         // this lane's class, real plane, tokens 32c..
         tmem_ld_32x32b_x32(trow + BM + 32 * c, v);    // imaginary plane
