@@ -242,7 +242,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         tmem_ld_32x32b_x32(trow + BM + 32 * c, v);    // imaginary plane
         tmem_wait_ld();
         // lane j < 16 (Br) takes tokens 32c + 0..15, lane j >= 16 (Bi) tokens 32c + 16..31;
-        // each gets the other class's values of its tokens from lane j ^ 16
+        // each gets the other class's values of its tokens from lane j ^ 16.  This lane's y
+        // entries are read first, then updated and written back, so the 16 read-add-write
+        // chains overlap.
+        const int tok0 = 32 * c + (imag ? 16 : 0);
+        float* yre = ys + tok0 * BN + o;
+        float* yim = ys + BM * BN + tok0 * BN + o;
+        float cre[16], cim[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          cre[i] = yre[i * BN];
+          cim[i] = yim[i * BN];
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float mu_lo = __uint_as_float(u[i]), mv_lo = __uint_as_float(v[i]);
@@ -253,11 +264,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           const float mu = imag ? mu_hi : mu_lo, mv = imag ? mv_hi : mv_lo;
           const float P_rr = imag ? pu : mu, P_ri = imag ? pv : mv;
           const float P_ir = imag ? mu : pu, P_ii = imag ? mv : pv;
-          const int tok = 32 * c + (imag ? 16 : 0) + i;
-          float* yre = ys + tok * BN + o;
-          float* yim = ys + BM * BN + tok * BN + o;
-          *yre += hr * P_rr + sgn * hi * P_ii;
-          *yim += hi * P_ir - sgn * hr * P_ri;
+          cre[i] += hr * P_rr + sgn * hi * P_ii;
+          cim[i] += hi * P_ir - sgn * hr * P_ri;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          yre[i * BN] = cre[i];
+          yim[i * BN] = cim[i];
         }
       }
       tc_fence_before();
