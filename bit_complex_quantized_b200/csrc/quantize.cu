@@ -123,15 +123,17 @@ __device__ __forceinline__ void block_sum3(double& a, double& b, unsigned long l
 // summed in float32 (at most 3 roundings of a sum of non-negative terms: below
 // 2e-7 relative) and that sum is added to the thread's float64 class sums.
 // Returns the code byte.
-template <int PREV>
+// kChecked: some entry of this thread is NaN or infinite (rare): entries that are
+// not finite are taken as 0.  Otherwise no per-entry test is made.
+template <int PREV, bool kChecked>
 __device__ __forceinline__ uint32_t quad_code(const float (&wr)[4], const float (&wi)[4], const uint32_t (&prev)[8],
-                                              const double (&sr)[8], const double (&si)[8], bool checked,
-                                              double& S_re, double& S_im) {
+                                              const double (&sr)[8], const double (&si)[8], double& S_re,
+                                              double& S_im) {
   uint32_t byte = 0;
   float q_re = 0.0f, q_im = 0.0f;
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    const bool fin = !checked || (isfinite(wr[e]) && isfinite(wi[e]));
+    const bool fin = !kChecked || (isfinite(wr[e]) && isfinite(wi[e]));
     uint32_t k;
     float v;
     if (PREV == 0) {
@@ -206,7 +208,8 @@ __global__ void __launch_bounds__(kQThreads) quant_stage_kernel(const __grid_con
   for (int q = 0; q < kQuadsPerThread; ++q) {
     const int64_t quad = quad0 + 32 * q;
     if (quad >= T.nquads) break;
-    const uint32_t byte = quad_code<PREV>(wr[q], wi[q], prev[q], sr, si, bad, S_re, S_im);
+    const uint32_t byte = bad ? quad_code<PREV, true>(wr[q], wi[q], prev[q], sr, si, S_re, S_im)
+                              : quad_code<PREV, false>(wr[q], wi[q], prev[q], sr, si, S_re, S_im);
     C_re += 4u - (uint32_t)__popc(byte & 0x55u);
     T.codes[(int64_t)PREV * T.nquads + quad] = (uint8_t)byte;
   }
