@@ -219,9 +219,9 @@ class Block:
         return len(self.cfg.layers) + 2 + gemv + len(self.gemm_layers)
 
 
-def oracle_decode_sample(seconds_budget=10.0, rows_per_layer=64, max_reps=50):
-    """The fp64 oracle's decode product on a row sample of the block (CPU), in GB/s of codes.
-    Codes come from the C oracle's quantizer run on the same row sample (setup, untimed)."""
+def oracle_sample_layers(rows_per_layer):
+    """A row sample of the block for the fp64 oracle: codes from the C oracle's quantizer on the
+    sampled rows (setup, untimed), and the block's activations."""
     import oracle as O
     from oracle import cref
     cfg = W.config("c3")
@@ -239,13 +239,19 @@ def oracle_decode_sample(seconds_budget=10.0, rows_per_layer=64, max_reps=50):
         xr, xi = W.activations(cfg, i, 1)
         layers.append((cu, su, cw, sw, W.bf16_to_f32_numpy(xr), W.bf16_to_f32_numpy(xi)))
     nbytes = sum(2 * cfg.T * rows_per_layer * l.K // 4 for l in cfg.layers)
+    return layers, nbytes
+
+
+def oracle_decode_time(layers, nbytes, rows_per_layer, seconds_budget):
+    """Times the fp64 oracle's decode product on the sample for about `seconds_budget` (CPU)."""
+    import oracle as O
     reps, t0 = 0, time.perf_counter()
     while True:
         for (cu, su, cw, sw, xr, xi) in layers:
             O.product(cu, su, cw, sw, xr, xi)
         reps += 1
         el = time.perf_counter() - t0
-        if el >= seconds_budget or reps >= max_reps:
+        if el >= seconds_budget:
             break
     try:
         from threadpoolctl import threadpool_info
@@ -255,6 +261,31 @@ def oracle_decode_sample(seconds_budget=10.0, rows_per_layer=64, max_reps=50):
     return {"value": nbytes * reps / el / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": f"fp64 NumPy oracle decode product, B=1, {rows_per_layer} sampled rows of each of the 7 "
                       f"layers, U+W, T=2 ({nbytes / 1e6:.2f} MB of codes per rep), {reps} reps in {el:.1f} s"}
+
+
+def oracle_decode_sample(seconds_budget=12.0, rows_per_layer=256):
+    layers, nbytes = oracle_sample_layers(rows_per_layer)
+    return oracle_decode_time(layers, nbytes, rows_per_layer, seconds_budget)
+
+
+# ---------------------------------------------------------------- decode at B = 16
+def decode_b16(block, reps=20):
+    """The block's decode product at B = 16 (the bf16 mma.sync path), after an L2 flush, through
+    the same grouped call; reported beside the step, not part of it."""
+    layers = block._layers(block.cfg, 16)
+    times = []
+    for i in range(reps + 3):
+        block.flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        Q.ifq_gemv(layers, block.T, 16, dev_status=block.status)
+        b.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            times.append(a.elapsed_time(b) * 1e-3)
+    t = statistics.median(times)
+    nbytes = block.gemv_bytes(16)
+    return {"us": t * 1e6, "algorithmic_bytes": nbytes, "GBps": nbytes / t / 1e9}
 
 
 # ---------------------------------------------------------------- dense comparator
@@ -395,6 +426,9 @@ def run_ours(args):
     cpu = None
     if rank == 0 and ws == 1 and not args.skip_cpu_baseline:
         cpu = oracle_decode_sample(seconds_budget=args.cpu_seconds)
+    b16 = decode_b16(block) if rank == 0 else None
+    if b16 is not None:
+        b16["frac_of_hbm"] = b16["GBps"] / float(peaks()[0]["hbm_gbs"])
     dense = None
     if rank == 0 and not args.skip_dense:
         dense = dense_comparator(block)
@@ -447,6 +481,7 @@ def run_ours(args):
         "kernels": kernels,
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "decode_b16": b16,
         "dense_bf16_comparator": dense,
         "gpu_launches": block.launches_per_step() * args.steps,
         "clocks": clk,
@@ -460,9 +495,10 @@ def run_reference(args):
     if rank != 0:
         return
     reps = []
-    for i in range(args.warmup + args.steps):
-        r = oracle_decode_sample(seconds_budget=args.cpu_seconds / max(1, args.steps), rows_per_layer=32,
-                                 max_reps=5)
+    rows = 128
+    layers, nbytes = oracle_sample_layers(rows)
+    for i in range(args.warmup + args.steps):  # each step: a bounded sample of the block's decode product
+        r = oracle_decode_time(layers, nbytes, rows, seconds_budget=min(5.0, 60.0 / max(1, args.steps)))
         if i >= args.warmup:
             reps.append(r)
     v = statistics.mean(r["value"] for r in reps)
@@ -578,7 +614,7 @@ def main():
     ap.add_argument("--case", choices=["gemv", "gemm", "quant", "convert"], default=None)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--workload", choices=["c3", "c5"], default="c5", help="layer set of --case gemv")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-dense", action="store_true", help="skip the cuBLAS bf16 dense comparator")
     args = ap.parse_args()
