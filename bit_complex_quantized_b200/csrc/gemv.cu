@@ -1,10 +1,11 @@
-// Decode product y = sum_t (U_hat_t x + W_hat_t conj(x)) for B = 1..16 tokens
+// Decode product y = sum_t (U_hat_t x + W_hat_t conj(x)) for B = 2..16 tokens
 // ("Fairy2i write-up" §2.1, §4.2; "iFairy article" §二.2; "iFairy talk notes" §2.3.1).
 //
-// Work split: one CTA of 4 warps per 16-row tile of one layer; warp w takes the
-// 256-code K-chunks c = w, w+4, ... of every (stage, branch) code matrix, and
-// the four warps' partial outputs are summed in a fixed order through shared
-// memory, so results are bit-reproducible.
+// Work split: one CTA of 4 warps per 64-row block of one layer (warp w: rows
+// 16w..16w+15); blocks of longer layers are numbered first so they start first.
+// The CTA walks K in chunks of 256 positions: the chunk of x for all B tokens
+// (both planes, bf16) is staged once in shared memory, and every warp uses it
+// for its 16 rows and every (stage, branch) code matrix.
 //
 // Per code, no multiplication by a weight happens: the 2-bit code is turned
 // into a pair of exact bf16 operands for the two axis classes,
@@ -19,18 +20,25 @@
 //     P_rr = sum Br x_re, P_ri = sum Br x_im, P_ir = sum Bi x_re, P_ii = sum Bi x_im
 // with exact products (+-2 times bf16) and float32 accumulation.  Columns of
 // the MMA are (token, plane) pairs: column 2b = x_re of token b, 2b+1 = x_im.
-// The epilogue applies the scales once per (stage, branch):
+// After each chunk the scales of each (stage, branch) are applied:
 //     U:  y_re += s_re P_rr - s_im P_ii,   y_im += s_re P_ri + s_im P_ir
 //     W:  y_re += s_re P_rr + s_im P_ii,   y_im += s_im P_ir - s_re P_ri
-// (times 1/2 for the operand encoding).
+// (times 1/2 for the operand encoding).  All sums run in a fixed order, so
+// results are bit-reproducible.
 #include "ifq_common.cuh"
 #include "ifq_internal.h"
 
 namespace ifq {
 namespace {
 
-constexpr int kWarpsPerTile = 4;
+constexpr int kWarps = 4;
+constexpr int kRowsPerBlock = 16 * kWarps;
 constexpr int kChunkCodes = 256;  // codes per row per chunk: 4 threads x 16 bytes
+// A staged (token, plane) row holds the chunk's 256 positions as 4 segments of 64 (one per
+// lane group tq), each followed by 8 bf16 of padding: 288 bf16 = 576 bytes.  The four
+// segments of a row, and the two planes, then fall on distinct banks.
+constexpr int kSeg = 64 + 8;
+constexpr int kXRow = 4 * kSeg;
 
 struct GemvLayerArg {
   const uint8_t* codes[2];
@@ -39,25 +47,25 @@ struct GemvLayerArg {
   float* y[2];           // re, im
   int64_t N;
   int64_t K;
-  int64_t tile_begin;
+  int64_t block_begin;
   int nbranch;
   int pad;
 };
 
 struct GemvParams {
   GemvLayerArg L[IFQ_MAX_GROUP];
+  int order[IFQ_MAX_GROUP];  // layers by decreasing K: block numbering order
   int count;
   int T;
   int B;
   int pad;
-  int64_t total_tiles;
+  int64_t total_blocks;
   uint32_t* status;
 };
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -71,80 +79,72 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   return v;
 }
 
-// NT: MMA n-tiles (8 columns = 4 tokens each); MI: code matrices handled per pass.
+// NT: MMA n-tiles (8 columns = 4 tokens each); MI: code matrices per pass over a chunk.
 template <int NT, int MI>
-__global__ void __launch_bounds__(32 * kWarpsPerTile) gemv_kernel(const __grid_constant__ GemvParams p) {
-  const int64_t tile = blockIdx.x;
-  int li = 0;
-  while (li + 1 < p.count && tile >= p.L[li + 1].tile_begin) ++li;
-  const GemvLayerArg& L = p.L[li];
+__global__ void __launch_bounds__(32 * kWarps) gemv_kernel(const __grid_constant__ GemvParams p) {
+  __shared__ __align__(16) uint16_t xs[4 * NT][2][kXRow];  // [token][plane][position in chunk]
+  const int64_t blk = blockIdx.x;
+  int oi = 0;
+  while (oi + 1 < p.count && blk >= p.L[p.order[oi + 1]].block_begin) ++oi;
+  const GemvLayerArg& L = p.L[p.order[oi]];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
-  const int64_t row0 = (tile - L.tile_begin) * 16;
+  const int64_t row0 = (blk - L.block_begin) * kRowsPerBlock + 16 * warp;
   const int64_t rowA = row0 + g, rowB = row0 + g + 8;
   const bool okA = rowA < L.N, okB = rowB < L.N;
   const int64_t K = L.K;
   const int64_t rb = K >> 2;  // bytes per code row
   const int nmat = p.T * L.nbranch;
   const int nchunks = (int)((K + kChunkCodes - 1) / kChunkCodes);
-
-  // B-operand column owned by this thread in n-tile nt: token nt*4 + g/2, plane g&1.
-  const uint16_t* xcol[NT];
-  bool xok[NT];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int tok = nt * 4 + (g >> 1);
-    xok[nt] = tok < p.B;
-    xcol[nt] = L.x[g & 1] + (int64_t)(xok[nt] ? tok : 0) * K;
-  }
+  const int ntok = 4 * NT;
 
   float yr[NT][2], yi[NT][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) yr[nt][0] = yr[nt][1] = yi[nt][0] = yi[nt][1] = 0.0f;
 
-  for (int m0 = 0; m0 < nmat; m0 += MI) {
-    float acc[MI][NT][2][4];
-#pragma unroll
-    for (int i = 0; i < MI; ++i)
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int c = 0; c < 2; ++c) acc[i][nt][c][0] = acc[i][nt][c][1] = acc[i][nt][c][2] = acc[i][nt][c][3] = 0.f;
-
-    const uint8_t* mrowA[MI];
-    const uint8_t* mrowB[MI];
-#pragma unroll
-    for (int i = 0; i < MI; ++i) {
-      const int m = m0 + i;
-      const int t = m / L.nbranch, br = m % L.nbranch;
-      const uint8_t* base = L.codes[br] + (int64_t)t * L.N * rb;
-      mrowA[i] = base + (okA ? rowA : 0) * rb;
-      mrowB[i] = base + (okB ? rowB : 0) * rb;
+  for (int c = 0; c < nchunks; ++c) {
+    const int64_t kc = (int64_t)c * kChunkCodes;
+    const int klen = (int)(K - kc < kChunkCodes ? K - kc : kChunkCodes);  // multiple of 64
+    // ---- stage x of the chunk: [token][plane][256] bf16; tokens past B and positions past K are 0
+    __syncthreads();  // the previous chunk's fragments are no longer read
+    for (int e = threadIdx.x; e < ntok * 2 * (kChunkCodes / 8); e += 32 * kWarps) {
+      const int seg = e % (kChunkCodes / 8), pl = (e / (kChunkCodes / 8)) & 1, tok = e / (2 * (kChunkCodes / 8));
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (tok < p.B && seg * 8 < klen) v = __ldg(reinterpret_cast<const uint4*>(L.x[pl] + (int64_t)tok * K + kc) + seg);
+      *reinterpret_cast<uint4*>(&xs[tok][pl][(seg >> 3) * kSeg + (seg & 7) * 8]) = v;
     }
+    __syncthreads();
 
-    for (int c = warp; c < nchunks; c += kWarpsPerTile) {
-      const int64_t pos0 = (int64_t)c * kChunkCodes + tq * 64;  // this thread's 64 K positions
-      const bool kok = pos0 < K;                                // K % 64 == 0: all-or-nothing
+    // B-operand column of this thread in n-tile nt: token nt*4 + g/2, plane g&1.
+    const int p0 = tq * 64;  // this thread's 64 positions of the chunk
+    const bool kok = p0 < klen;
+    for (int m0 = 0; m0 < nmat; m0 += MI) {
+      float acc[MI][NT][2][4];
+#pragma unroll
+      for (int i = 0; i < MI; ++i)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int cl = 0; cl < 2; ++cl) acc[i][nt][cl][0] = acc[i][nt][cl][1] = acc[i][nt][cl][2] = acc[i][nt][cl][3] = 0.f;
       uint4 wa[MI], wb[MI];
 #pragma unroll
       for (int i = 0; i < MI; ++i) {
-        wa[i] = (kok && okA) ? ld_nc_v4(mrowA[i] + (pos0 >> 2)) : make_uint4(0, 0, 0, 0);
-        wb[i] = (kok && okB) ? ld_nc_v4(mrowB[i] + (pos0 >> 2)) : make_uint4(0, 0, 0, 0);
+        const int m = m0 + i < nmat ? m0 + i : nmat - 1;
+        const int t = m / L.nbranch, br = m % L.nbranch;
+        const uint8_t* base = L.codes[br] + (int64_t)t * L.N * rb + ((kc + p0) >> 2);
+        wa[i] = (kok && okA && m0 + i < nmat) ? ld_nc_v4(base + rowA * rb) : make_uint4(0, 0, 0, 0);
+        wb[i] = (kok && okB && m0 + i < nmat) ? ld_nc_v4(base + rowB * rb) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
         uint32_t X[NT][8];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          if (kok && xok[nt]) {
-            const uint4 lo = __ldg(reinterpret_cast<const uint4*>(xcol[nt] + pos0 + 16 * w));
-            const uint4 hi = __ldg(reinterpret_cast<const uint4*>(xcol[nt] + pos0 + 16 * w + 8));
-            X[nt][0] = lo.x; X[nt][1] = lo.y; X[nt][2] = lo.z; X[nt][3] = lo.w;
-            X[nt][4] = hi.x; X[nt][5] = hi.y; X[nt][6] = hi.z; X[nt][7] = hi.w;
-          } else {
-#pragma unroll
-            for (int q = 0; q < 8; ++q) X[nt][q] = 0u;
-          }
+          const uint16_t* xp = &xs[nt * 4 + (g >> 1)][g & 1][tq * kSeg + 16 * w];
+          const uint4 lo = *reinterpret_cast<const uint4*>(xp);
+          const uint4 hi = *reinterpret_cast<const uint4*>(xp + 8);
+          X[nt][0] = lo.x; X[nt][1] = lo.y; X[nt][2] = lo.z; X[nt][3] = lo.w;
+          X[nt][4] = hi.x; X[nt][5] = hi.y; X[nt][6] = hi.z; X[nt][7] = hi.w;
         }
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
@@ -172,65 +172,47 @@ __global__ void __launch_bounds__(32 * kWarpsPerTile) gemv_kernel(const __grid_c
           }
         }
       }
-    }
 
-    // Apply the scales of each matrix (halved: operands carry a factor 2).
+      // Apply the scales of each matrix (halved: operands carry a factor 2).
 #pragma unroll
-    for (int i = 0; i < MI; ++i) {
-      const int m = m0 + i;
-      const int t = m / L.nbranch, br = m % L.nbranch;
-      const float hr = 0.5f * __ldg(L.scales[br] + 2 * t);
-      const float hi = 0.5f * __ldg(L.scales[br] + 2 * t + 1);
+      for (int i = 0; i < MI; ++i) {
+        const int m = m0 + i;
+        if (m >= nmat) break;
+        const int t = m / L.nbranch, br = m % L.nbranch;
+        const float hr = 0.5f * __ldg(L.scales[br] + 2 * t);
+        const float hi = 0.5f * __ldg(L.scales[br] + 2 * t + 1);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const float* Pr = acc[i][nt][0];  // {P_rr g, P_ri g, P_rr g+8, P_ri g+8}
-        const float* Pi = acc[i][nt][1];  // {P_ir g, P_ii g, P_ir g+8, P_ii g+8}
-        if (br == 0) {
-          yr[nt][0] += hr * Pr[0] - hi * Pi[1];
-          yi[nt][0] += hr * Pr[1] + hi * Pi[0];
-          yr[nt][1] += hr * Pr[2] - hi * Pi[3];
-          yi[nt][1] += hr * Pr[3] + hi * Pi[2];
-        } else {
-          yr[nt][0] += hr * Pr[0] + hi * Pi[1];
-          yi[nt][0] += hi * Pi[0] - hr * Pr[1];
-          yr[nt][1] += hr * Pr[2] + hi * Pi[3];
-          yi[nt][1] += hi * Pi[2] - hr * Pr[3];
+        for (int nt = 0; nt < NT; ++nt) {
+          const float* Pr = acc[i][nt][0];  // {P_rr g, P_ri g, P_rr g+8, P_ri g+8}
+          const float* Pi = acc[i][nt][1];  // {P_ir g, P_ii g, P_ir g+8, P_ii g+8}
+          if (br == 0) {
+            yr[nt][0] += hr * Pr[0] - hi * Pi[1];
+            yi[nt][0] += hr * Pr[1] + hi * Pi[0];
+            yr[nt][1] += hr * Pr[2] - hi * Pi[3];
+            yi[nt][1] += hr * Pr[3] + hi * Pi[2];
+          } else {
+            yr[nt][0] += hr * Pr[0] + hi * Pi[1];
+            yi[nt][0] += hi * Pi[0] - hr * Pr[1];
+            yr[nt][1] += hr * Pr[2] + hi * Pi[3];
+            yi[nt][1] += hi * Pi[2] - hr * Pr[3];
+          }
         }
       }
     }
   }
 
-  // Sum the warps' K-slices in a fixed order and store.
-  __shared__ float red[kWarpsPerTile][NT * 4][32];
+  // Columns 2tq, 2tq+1 of n-tile nt are token nt*4 + tq, planes re / im: rows g, g+8.
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    red[warp][nt * 4 + 0][lane] = yr[nt][0];
-    red[warp][nt * 4 + 1][lane] = yi[nt][0];
-    red[warp][nt * 4 + 2][lane] = yr[nt][1];
-    red[warp][nt * 4 + 3][lane] = yi[nt][1];
-  }
-  __syncthreads();
-  if (warp == 0) {
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      float v[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float s = red[0][nt * 4 + q][lane];
-#pragma unroll
-        for (int w = 1; w < kWarpsPerTile; ++w) s += red[w][nt * 4 + q][lane];
-        v[q] = s;
+    const int tok = nt * 4 + tq;
+    if (tok < p.B) {
+      if (okA) {
+        L.y[0][(int64_t)tok * L.N + rowA] = yr[nt][0];
+        L.y[1][(int64_t)tok * L.N + rowA] = yi[nt][0];
       }
-      const int tok = nt * 4 + tq;
-      if (tok < p.B) {
-        if (okA) {
-          L.y[0][(int64_t)tok * L.N + rowA] = v[0];
-          L.y[1][(int64_t)tok * L.N + rowA] = v[1];
-        }
-        if (okB) {
-          L.y[0][(int64_t)tok * L.N + rowB] = v[2];
-          L.y[1][(int64_t)tok * L.N + rowB] = v[3];
-        }
+      if (okB) {
+        L.y[0][(int64_t)tok * L.N + rowB] = yr[nt][1];
+        L.y[1][(int64_t)tok * L.N + rowB] = yi[nt][1];
       }
     }
   }
@@ -238,19 +220,8 @@ __global__ void __launch_bounds__(32 * kWarpsPerTile) gemv_kernel(const __grid_c
 
 template <int NT, int MI>
 cudaError_t launch_nt_mi(const GemvParams& p, cudaStream_t s) {
-  gemv_kernel<NT, MI><<<(unsigned)p.total_tiles, 32 * kWarpsPerTile, 0, s>>>(p);
+  gemv_kernel<NT, MI><<<(unsigned)p.total_blocks, 32 * kWarps, 0, s>>>(p);
   return cudaGetLastError();
-}
-
-// Several matrices per pass only pay off with one n-tile (B <= 4); with more
-// n-tiles the accumulators already fill the register file.
-cudaError_t launch_nt1(const GemvParams& p, int mi, cudaStream_t s) {
-  switch (mi) {
-    case 4: return launch_nt_mi<1, 4>(p, s);
-    case 3: return launch_nt_mi<1, 3>(p, s);
-    case 2: return launch_nt_mi<1, 2>(p, s);
-    default: return launch_nt_mi<1, 1>(p, s);
-  }
 }
 
 }  // namespace
@@ -262,7 +233,6 @@ cudaError_t launch_gemv(const ifq_layer* Ls, int count, int T, int B, uint32_t* 
   p.T = T;
   p.B = B;
   p.status = dev_status;
-  int64_t tiles = 0;
   for (int i = 0; i < count; ++i) {
     GemvLayerArg& a = p.L[i];
     a.codes[0] = Ls[i].codes_u;
@@ -276,30 +246,29 @@ cudaError_t launch_gemv(const ifq_layer* Ls, int count, int T, int B, uint32_t* 
     a.y[1] = Ls[i].y_im;
     a.N = Ls[i].N;
     a.K = Ls[i].K;
-    a.tile_begin = tiles;
-    tiles += (Ls[i].N + 15) / 16;
+    p.order[i] = i;
   }
-  p.total_tiles = tiles;
-  if (tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  const int NT = (2 * B + 7) / 8;
-  // Matrices per pass: the largest of 4, 3, 2 that divides every layer's
-  // (stage, branch) matrix count, so that one activation-fragment load serves them all.
-  int mi = 1;
-  if (NT == 1) {
-    for (int c : {4, 3, 2}) {
-      bool ok = true;
-      for (int i = 0; i < count; ++i) ok &= (T * p.L[i].nbranch) % c == 0;
-      if (ok) {
-        mi = c;
-        break;
-      }
+  // Longest rows first (stable): their blocks are launched first.
+  for (int i = 1; i < count; ++i)
+    for (int j = i; j > 0 && p.L[p.order[j]].K > p.L[p.order[j - 1]].K; --j) {
+      const int t = p.order[j];
+      p.order[j] = p.order[j - 1];
+      p.order[j - 1] = t;
     }
+  int64_t blocks = 0;
+  for (int i = 0; i < count; ++i) {
+    GemvLayerArg& a = p.L[p.order[i]];
+    a.block_begin = blocks;
+    blocks += (a.N + kRowsPerBlock - 1) / kRowsPerBlock;
   }
+  p.total_blocks = blocks;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  const int NT = (2 * B + 7) / 8;
   switch (NT) {
-    case 1: return launch_nt1(p, mi, s);
-    case 2: return launch_nt_mi<2, 1>(p, s);
-    case 3: return launch_nt_mi<3, 1>(p, s);
-    default: return launch_nt_mi<4, 1>(p, s);
+    case 1: return launch_nt_mi<1, 4>(p, s);
+    case 2: return launch_nt_mi<2, 2>(p, s);
+    case 3: return launch_nt_mi<3, 2>(p, s);
+    default: return launch_nt_mi<4, 2>(p, s);
   }
 }
 
