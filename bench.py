@@ -326,23 +326,37 @@ def dense_comparator(block, reps=20):
 
 # ---------------------------------------------------------------- e2e
 def e2e_decode(block, steps, warmup):
-    """Decode GEMV through the public API with host buffers: per step, pinned host -> device
-    copy of every layer's x, the grouped GEMV, device -> host copy of every y."""
+    """Decode GEMV through the public API with host buffers: per step, one pinned host -> device
+    copy of every layer's x (packed in one buffer), the grouped GEMV, and one device -> host copy
+    of every y (packed in one buffer)."""
     dev = block.dev
-    host_x = [(L["x_re"].cpu().pin_memory(), L["x_im"].cpu().pin_memory()) for L in block.gemv_layers]
-    host_y = [(torch.empty_like(L["y_re"], device="cpu").pin_memory(),
-               torch.empty_like(L["y_im"], device="cpu").pin_memory()) for L in block.gemv_layers]
-    h2d = sum(a.numel() * a.element_size() + b.numel() * b.element_size() for a, b in host_x)
-    d2h = sum(a.numel() * a.element_size() + b.numel() * b.element_size() for a, b in host_y)
+    xs = [t for L in block.gemv_layers for t in (L["x_re"], L["x_im"])]
+    ys = [t for L in block.gemv_layers for t in (L["y_re"], L["y_im"])]
+    x_dev = torch.empty(sum(t.numel() for t in xs), dtype=torch.bfloat16, device=dev)
+    y_dev = torch.empty(sum(t.numel() for t in ys), dtype=torch.float32, device=dev)
+
+    def views(buf, like):
+        out, off = [], 0
+        for t in like:
+            out.append(buf[off:off + t.numel()].view(t.shape))
+            off += t.numel()
+        return out
+    xv, yv = views(x_dev, xs), views(y_dev, ys)
+    layers = []
+    for i, L in enumerate(block.gemv_layers):
+        d = dict(L)
+        d["x_re"], d["x_im"], d["y_re"], d["y_im"] = xv[2 * i], xv[2 * i + 1], yv[2 * i], yv[2 * i + 1]
+        layers.append(d)
+    prepared = Q.LayerSet(layers)
+    x_host = torch.cat([t.flatten().cpu() for t in xs]).pin_memory()
+    y_host = torch.empty(y_dev.numel(), dtype=torch.float32).pin_memory()
+    h2d = x_host.numel() * x_host.element_size()
+    d2h = y_host.numel() * y_host.element_size()
 
     def one():
-        for L, (xr, xi) in zip(block.gemv_layers, host_x):
-            L["x_re"].copy_(xr, non_blocking=True)
-            L["x_im"].copy_(xi, non_blocking=True)
-        Q.ifq_gemv(block.gemv_layers, block.T, block.B, workspace=block.gemv_ws, dev_status=block.status)
-        for L, (yr, yi) in zip(block.gemv_layers, host_y):
-            yr.copy_(L["y_re"], non_blocking=True)
-            yi.copy_(L["y_im"], non_blocking=True)
+        x_dev.copy_(x_host, non_blocking=True)
+        Q.ifq_gemv(prepared, block.T, block.B, workspace=block.gemv_ws, dev_status=block.status)
+        y_host.copy_(y_dev, non_blocking=True)
 
     times = []
     for i in range(warmup + steps):

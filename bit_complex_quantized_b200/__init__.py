@@ -13,6 +13,7 @@ from ._lib import (  # noqa: F401
     IFQ_MAX_STAGES,
     IFQ_QUANT_STATIC_SCRATCH_BYTES,
     IfqError,
+    LayerSet,
     LIB_PATH,
     ifq_gemm,
     ifq_gemv,

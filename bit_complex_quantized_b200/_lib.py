@@ -153,8 +153,25 @@ def _layers(layers):
     return arr
 
 
+class LayerSet:
+    """Layer descriptors marshalled once, for a caller that repeats the same grouped call
+    (the tensors must stay alive and in place).  Accepted wherever a list of layer dicts is."""
+
+    def __init__(self, layers):
+        self.layers = list(layers)
+        self.array = _layers(self.layers)
+
+    def __len__(self):
+        return len(self.layers)
+
+
+def _as_array(layers):
+    return (layers.array, len(layers)) if isinstance(layers, LayerSet) else (_layers(layers), len(layers))
+
+
 def ifq_gemv_workspace_bytes(layers, T, B):
-    return int(load().ifq_gemv_workspace_bytes(_layers(layers), len(layers), T, B))
+    arr, n = _as_array(layers)
+    return int(load().ifq_gemv_workspace_bytes(arr, n, T, B))
 
 
 def ifq_gemv(layers, T, B, workspace=None, dev_status=None, stream=None, workspace_bytes=None):
@@ -164,13 +181,14 @@ def ifq_gemv(layers, T, B, workspace=None, dev_status=None, stream=None, workspa
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     if workspace_bytes is not None:
         nbytes = workspace_bytes
-    _check(load().ifq_gemv(_layers(layers), len(layers), T, B, _ptr(workspace), nbytes, _ptr(dev_status),
-                           _stream(stream)))
+    arr, n = _as_array(layers)
+    _check(load().ifq_gemv(arr, n, T, B, _ptr(workspace), nbytes, _ptr(dev_status), _stream(stream)))
 
 
 def ifq_gemm(layers, T, M, dev_status=None, stream=None):
     """As ifq_gemv with x [M][K] and y [M][N]."""
-    _check(load().ifq_gemm(_layers(layers), len(layers), T, M, _ptr(dev_status), _stream(stream)))
+    arr, n = _as_array(layers)
+    _check(load().ifq_gemm(arr, n, T, M, _ptr(dev_status), _stream(stream)))
 
 
 # Raw entry point for callers that build ctypes descriptors themselves.

@@ -124,3 +124,16 @@ def test_convert_argument_errors():
     assert lib.ifq_widely_linear_from_real(FAKE, 3, 4, FAKE, FAKE, FAKE, FAKE, None) == 2
     assert lib.ifq_widely_linear_from_real(FAKE, 4, 0, FAKE, FAKE, FAKE, FAKE, None) == 2
     assert lib.ifq_widely_linear_from_real(FAKE, 4, 4, FAKE + 4, FAKE, FAKE, FAKE, None) == 3
+
+
+def test_layerset_marshals_the_same_descriptors():
+    import torch
+    t = lambda *s: torch.zeros(*s, dtype=torch.float32)  # noqa: E731
+    layers = [dict(codes_u=torch.zeros(2, 8, 16, dtype=torch.uint8), scales_u=t(2, 2), codes_w=None, scales_w=None,
+                   N=8, K=64, x_re=t(1, 64), x_im=t(1, 64), y_re=t(1, 8), y_im=t(1, 8)) for _ in range(3)]
+    a = L._layers(layers)
+    b = Q.LayerSet(layers)
+    assert len(b) == 3
+    for x, y in zip(a, b.array):
+        for f, _ in L.Layer._fields_:
+            assert getattr(x, f) == getattr(y, f)

@@ -416,3 +416,21 @@ def test_max_group_of_32_layers():
         assert int(st.item()) == 0
         for d, (cun, sun, cwn, swn, xrn, xin) in zip(descs, ref):
             check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cun, sun, cwn, swn, xrn, xin)
+
+
+def test_prepared_layer_set_gives_the_same_product():
+    """A LayerSet (descriptors marshalled once) and a list of layer dicts run the same call."""
+    rng = np.random.default_rng(515)
+    N, K, T = 80, 320, 2
+    ws = [_rand_complex(rng, N, K), _rand_complex(rng, N, K, 0.03)]
+    outs = gpu_quantize([(to_dev(a), to_dev(b)) for a, b in ws], T)
+    for B in (1, 3):
+        xr = torch.from_numpy(rng.standard_normal((B, K)).astype(np.float32)).to(torch.bfloat16).to(DEV)
+        xi = torch.from_numpy(rng.standard_normal((B, K)).astype(np.float32)).to(torch.bfloat16).to(DEV)
+        d1 = layer_desc(outs[0][0], outs[0][1], outs[1][0], outs[1][1], xr, xi, N, K, B)
+        d2 = layer_desc(outs[0][0], outs[0][1], outs[1][0], outs[1][1], xr, xi, N, K, B)
+        run_gemv([d1], T, B)
+        wsz = max(16, Q.ifq_gemv_workspace_bytes(Q.LayerSet([d2]), T, B))
+        Q.ifq_gemv(Q.LayerSet([d2]), T, B, workspace=torch.zeros(wsz, dtype=torch.uint8, device=DEV))
+        torch.cuda.synchronize()
+        assert torch.equal(d1["y_re"], d2["y_re"]) and torch.equal(d1["y_im"], d2["y_im"])
