@@ -28,9 +28,8 @@
 // matrix), ordered tile by tile, and every warp of a persistent grid takes an
 // equal contiguous range of chunks (stream-K), so the load is balanced to one
 // chunk.  A warp walks its range in pieces (one tile, one matrix, one K block
-// at most), streams each piece's 16 code rows into a double-buffered shared
-// slot with cp.async.bulk (one row per lane, completion on an mbarrier), and
-// runs mma.sync m16n8k32 s8 (columns = plane x digit, exact int32
+// at most), streams each piece into a double-buffered shared slot (completion
+// on an mbarrier), and runs mma.sync m16n8k32 s8 (columns = plane x digit, exact int32
 // accumulation).  Per tile it keeps the float64 output sums in registers; a
 // tile split between warps leaves one partial per warp in the workspace, and
 // the last of them to arrive (atomic ticket) adds the partials in warp order
@@ -47,14 +46,18 @@ constexpr int kKBlock = 2048;                  // K positions per exponent block
 constexpr int kKsteps = kKBlock / 32;          // MMA k-steps per block (64)
 constexpr int kWarps = 4;                      // warps per CTA in the main kernel
 constexpr int kPieceChunks = 8;                // at most 8 chunks (256 K positions each) per piece: one K block
-constexpr int kSlotRow = 576;                  // bytes per code row in a slot (512 + 64 pad: conflict-free)
-constexpr int kSlotBytes = 16 * kSlotRow;      // one 16-row slot
+constexpr int kSlotBytes = 8192;               // one slot: 16 rows x 8 chunks x 64 bytes
 constexpr int kMainSmem = kWarps * 2 * kSlotBytes + kWarps * 2 * 8;
 constexpr int kPrepThreads = 128;                // one item (plane, position, 16-group) per thread of a chunk
 constexpr int kCtasPerSm = 3;
 static_assert(kPieceChunks * 256 == kKBlock, "a piece is at most one K block, and one run of the int32 sums");
 
+// Slot layouts.  Pieces inside a full K block arrive by one 4-D tensor copy as
+// [chunk][row][64 B] (lanes of a quarter warp read two adjacent 64-byte rows:
+// conflict-free).  Pieces of a row's last, partial block arrive by one bulk copy
+// per row as [row][512 B].
 struct I8Layer {
+  CUtensorMap tmap[2];    // per branch: (64 B, row of [T][N], chunk in block, full block), box 64 x 16 x 8 x 1
   const uint8_t* codes[2];
   const float* scales[2];
   const uint16_t* x[2];
@@ -72,10 +75,15 @@ struct I8Layer {
   int32_t blocks;         // K blocks
   int32_t nbranch;
   int32_t nch;            // 256-wide K chunks per row
+  int32_t nbf;            // full 2048-wide K blocks (streamed by tensor copies)
 };
 
+// Capacity kCap >= count: calls of up to 8 layers pass a small parameter block.
+template <int kCap>
 struct I8Params {
-  I8Layer L[IFQ_MAX_GROUP];
+  int64_t chunk_begin[kCap];  // copies of the layers' first chunk and first prep CTA, packed so that
+  int64_t prep_begin[kCap];   // the search for a layer touches one or two constant-cache lines
+  I8Layer L[kCap];
   int64_t total_chunks;
   int count;
   int T;
@@ -97,9 +105,10 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                : "memory");
 }
 
-__device__ __forceinline__ int find_layer_by(const I8Params& p, int64_t idx, bool prep) {
+template <class P>
+__device__ __forceinline__ int find_layer_by(const P& p, int64_t idx, bool prep) {
   int li = 0;
-  while (li + 1 < p.count && idx >= (prep ? p.L[li + 1].prep_begin : p.L[li + 1].chunk_begin)) ++li;
+  while (li + 1 < p.count && idx >= (prep ? p.prep_begin[li + 1] : p.chunk_begin[li + 1])) ++li;
   return li;
 }
 
@@ -108,7 +117,8 @@ __device__ __forceinline__ int find_layer_by(const I8Params& p, int64_t idx, boo
 // block's exponent, then writes the digit fragments of its own chunk and the
 // exact sum of v up to its chunk's end (prefix sums at chunk boundaries).  The
 // first CTA of a layer also zeroes the layer's tile tickets.
-__global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(const __grid_constant__ I8Params p) {
+template <class P>
+__global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(const __grid_constant__ P p) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ __align__(16) uint16_t xs[2][kKBlock];
   __shared__ unsigned int smax[kPrepThreads / 32];
@@ -240,13 +250,15 @@ __device__ __forceinline__ int piece_len(const I8Layer& L, int ch, int64_t gbegi
 }
 
 // The piece that starts at global chunk c (one division chain per warp, at its start).
-__device__ __forceinline__ Piece make_piece(const I8Params& p, int64_t c, int64_t c_hi) {
+template <class P>
+__device__ __forceinline__ Piece make_piece(const P& p, int64_t c, int64_t c_hi) {
   Piece pc;
   pc.li = find_layer_by(p, c, false);
   const I8Layer& L = p.L[pc.li];
   const int64_t tc = (int64_t)p.T * L.nbranch * L.nch;  // chunks per tile
-  const int64_t local = c - L.chunk_begin;
-  pc.tile = local / tc;
+  const int64_t local = c - p.chunk_begin[pc.li];
+  // 32-bit division when the operands fit (the usual case): far shorter than the 64-bit routine
+  pc.tile = (local | tc) < ((int64_t)1 << 32) ? (int64_t)((uint32_t)local / (uint32_t)tc) : local / tc;
   const int r = (int)(local - pc.tile * tc);
   pc.mat = r / L.nch;
   pc.ch = r - pc.mat * L.nch;
@@ -256,7 +268,8 @@ __device__ __forceinline__ Piece make_piece(const I8Params& p, int64_t c, int64_
 }
 
 // The piece after `pc` in chunk order (chunks, then matrices, then tiles, then layers).
-__device__ __forceinline__ Piece next_piece(const I8Params& p, const Piece& pc, int64_t c_hi) {
+template <class P>
+__device__ __forceinline__ Piece next_piece(const P& p, const Piece& pc, int64_t c_hi) {
   Piece n = pc;
   n.gbegin = pc.gbegin + pc.len;
   n.ch = pc.ch + pc.len;
@@ -283,7 +296,10 @@ __device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* addr, unsigne
 }
 
 // Warp w < W owns chunks [lo(w), lo(w+1)) with lo(w) = floor(w C / W); W <= C, so no range is empty.
-__device__ __forceinline__ int64_t range_lo(int64_t w, int64_t C, int64_t W) { return (w * C) / W; }
+__device__ __forceinline__ int64_t range_lo(int64_t w, int64_t C, int64_t W) {
+  const int64_t num = w * C;  // 32-bit division when the operands fit (the usual case)
+  return (num | W) < ((int64_t)1 << 32) ? (int64_t)((uint32_t)num / (uint32_t)W) : num / W;
+}
 
 
 // As imma_16832 with a zero accumulator input: starts a fresh sum without zeroing registers.
@@ -333,25 +349,55 @@ __device__ __forceinline__ void chunk_mma(int (&acc0)[4][4], int (&acc1)[4][4], 
   }
 }
 
-// Lanes 0..15 each copy one code row of the piece into the slot.
-__device__ __forceinline__ void issue_piece(const I8Params& p, const Piece& pc, uint32_t slot, uint64_t* bar,
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+      "[%6];" ::"r"(dst),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Where a piece's chunks sit in its slot.  In a full K block one tensor copy
+// brings chunks [ch, ch + 8) of the block, or, for a piece that starts at the
+// block start and stops early, chunks [ch + len - 8, ch + len): the coordinates
+// outside the block are zero-filled, not read.  So the piece's first chunk is
+// at chunk position p0 = 8 - len in that case, else 0.
+__device__ __forceinline__ bool piece_by_tensor(const I8Layer& L, const Piece& pc) { return (pc.ch >> 3) < L.nbf; }
+__device__ __forceinline__ int piece_p0(const Piece& pc) {
+  return ((pc.ch & 7) == 0 && pc.len < kPieceChunks) ? kPieceChunks - pc.len : 0;
+}
+
+// Put the piece's codes in flight into the slot.
+template <class P>
+__device__ __forceinline__ void issue_piece(const P& p, const Piece& pc, uint32_t slot, uint64_t* bar,
                                             int lane) {
   const I8Layer& L = p.L[pc.li];
   const int64_t row0 = pc.tile * 16;
+  const int t = L.nbranch == 2 ? pc.mat >> 1 : pc.mat, br = L.nbranch == 2 ? pc.mat & 1 : 0;
+  if (piece_by_tensor(L, pc)) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar, kSlotBytes);  // the whole box, zero-filled parts included
+      const int cib = piece_p0(pc) ? pc.len - kPieceChunks : (pc.ch & 7);
+      tma_load_4d(slot, &L.tmap[br], 0, (int)((int64_t)t * L.N + row0), cib, pc.ch >> 3, bar);
+    }
+    return;
+  }
+  // Last, partial K block of the rows: lanes 0..15 each copy one code row.
   const int rows = (int)(L.N - row0 < 16 ? L.N - row0 : 16);
   const int64_t kend = (int64_t)(pc.ch + pc.len) * 256 < L.K ? (int64_t)(pc.ch + pc.len) * 256 : L.K;
   const uint32_t bytes = (uint32_t)((kend - (int64_t)pc.ch * 256) >> 2);
   if (lane == 0) mbar_arrive_expect_tx(bar, bytes * (uint32_t)rows);
   __syncwarp();
   if (lane < rows) {
-    const int t = L.nbranch == 2 ? pc.mat >> 1 : pc.mat, br = L.nbranch == 2 ? pc.mat & 1 : 0;
     const int64_t rb = L.K >> 2;
     const uint8_t* src = L.codes[br] + ((int64_t)t * L.N + row0 + lane) * rb + (int64_t)pc.ch * 64;
-    bulk_g2s(slot + lane * kSlotRow, src, bytes, bar);
+    bulk_g2s(slot + lane * 512, src, bytes, bar);
   }
 }
 
-__global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_i8_kernel(const __grid_constant__ I8Params p) {
+template <class P>
+__global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_i8_kernel(const __grid_constant__ P p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
@@ -377,6 +423,9 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_i8_kernel(const 
   if (gw >= W) return;
   const int64_t c_lo = range_lo(gw, C, W), c_hi = range_lo(gw + 1, C, W);
 
+  // warm the TMA descriptor cache with this call's code maps, once per CTA
+  if (warp == 0 && lane < 2 * p.count && p.L[lane >> 1].nbf > 0 && (lane & 1) < p.L[lane >> 1].nbranch)
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&p.L[lane >> 1].tmap[lane & 1]) : "memory");
   int abort_flag = 0;
   uint32_t phases = 0u;  // bit s: parity of the next completion of slot s
   int s = 0;
@@ -437,12 +486,13 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_i8_kernel(const 
 
     const uint32_t slot = slots + s * kSlotBytes;  // shared-window address of this slot
     // Plain shared loads (ordered after the barrier wait above by its memory clobber).
-    const uint4* rowa = reinterpret_cast<const uint4*>(smem + (slot - slots0) + g * kSlotRow + tq * 16);
-    const uint4* rowb = rowa + 8 * kSlotRow / 16;
+    const uint8_t* sbase = smem + (slot - slots0) + tq * 16;
 
     int acc0[4][4], acc1[4][4];  // [position q][fragment reg]: the piece's int32 sums, started by chunk 0
     // Positions past K carry zero activation digits, so code bytes there (stale or not) add nothing.
-    if (cur.len == kPieceChunks) {
+    if (cur.len == kPieceChunks && piece_by_tensor(L, cur)) {  // a whole K block: chunk c at c * 1024
+      const uint4* rowa = reinterpret_cast<const uint4*>(sbase + g * 64);
+      const uint4* rowb = rowa + 512 / 16;
       uint4 Fc[4] = {F0[0], F0[1], F0[2], F0[3]};
 #pragma unroll
       for (int c = 0; c < kPieceChunks; ++c) {
@@ -454,20 +504,25 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_i8_kernel(const 
         if (c == 0)
           chunk_mma<true>(acc0, acc1, rowa, rowb, Fc);
         else
-          chunk_mma<false>(acc0, acc1, rowa + c * 4, rowb + c * 4, Fc);
+          chunk_mma<false>(acc0, acc1, rowa + c * 64, rowb + c * 64, Fc);
         if (c + 1 < kPieceChunks) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) Fc[k] = Fn[k];
         }
       }
     } else {
+      // tensor layout from chunk position p0 (strides 1024 per chunk, 64 per row) or row layout (64, 512)
+      const bool tens = piece_by_tensor(L, cur);
+      const int cstride = tens ? 1024 / 16 : 64 / 16, rstride = tens ? 64 : 512;
+      const uint4* rowa = reinterpret_cast<const uint4*>(sbase + (tens ? piece_p0(cur) * 1024 : 0) + g * rstride);
+      const uint4* rowb = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(rowa) + 8 * rstride);
       chunk_mma<true>(acc0, acc1, rowa, rowb, F0);
 #pragma unroll 1
       for (int c = 1; c < cur.len; ++c) {
         uint4 F[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) F[k] = __ldg(fr + c * 128 + k);
-        chunk_mma<false>(acc0, acc1, rowa + c * 4, rowb + c * 4, F);
+        chunk_mma<false>(acc0, acc1, rowa + c * cstride, rowb + c * cstride, F);
       }
     }
     __syncwarp();  // every lane is done with this slot before it is refilled
@@ -627,14 +682,18 @@ size_t layout_layers(const ifq_layer* Ls, int count, int T, WsLayout* out) {
 
 size_t gemv_i8_workspace_bytes(const ifq_layer* Ls, int count, int T) { return layout_layers(Ls, count, T, nullptr); }
 
-cudaError_t launch_gemv_i8(const ifq_layer* Ls, int count, int T, void* ws, uint32_t* dev_status, cudaStream_t s) {
+namespace {
+
+template <int kCap>
+cudaError_t launch_cap(const ifq_layer* Ls, int count, int T, void* ws, uint32_t* dev_status, cudaStream_t s) {
+  using P = I8Params<kCap>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(gemv_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMainSmem);
+    attr_err = cudaFuncSetAttribute(gemv_i8_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMainSmem);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  I8Params p;
+  P p;
   memset(&p, 0, sizeof(p));
   p.count = count;
   p.T = T;
@@ -665,15 +724,26 @@ cudaError_t launch_gemv_i8(const ifq_layer* Ls, int count, int T, void* ws, uint
     a.next = reinterpret_cast<int*>(base + lay[i].next);
     a.tickets = reinterpret_cast<unsigned int*>(base + lay[i].tick);
     a.nch = (int32_t)((a.K + 255) / 256);
-    a.chunk_begin = chunks;
-    a.prep_begin = preps;
+    a.nbf = (int32_t)(a.K / kKBlock);
+    if ((int64_t)T * a.N >= ((int64_t)1 << 31)) a.nbf = 0;  // rows beyond a tensor coordinate: row copies only
+    for (int b = 0; b < a.nbranch && a.nbf > 0; ++b) {
+      // (byte in chunk, row of [T][N], chunk in block, block): strides K/4, 64, 512 bytes
+      const uint64_t dims[4] = {64, (uint64_t)T * (uint64_t)a.N, 8, (uint64_t)a.nbf};
+      const uint64_t strides[3] = {(uint64_t)a.K / 4, 64, 512};
+      const uint32_t box[4] = {64, 16, 8, 1};
+      if (!encode_tiled_map(&a.tmap[b], CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, a.codes[b], dims, strides, box,
+                            CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    }
+    a.chunk_begin = p.chunk_begin[i] = chunks;
+    a.prep_begin = p.prep_begin[i] = preps;
     chunks += (int64_t)a.tiles * T * a.nbranch * a.nch;
     preps += (int64_t)a.blocks * 8;
   }
   p.total_chunks = chunks;
   if (chunks >= ((int64_t)1 << 40) || preps > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
 
-  gemv_prep_kernel<<<(unsigned)preps, kPrepThreads, 0, s>>>(p);
+  gemv_prep_kernel<P><<<(unsigned)preps, kPrepThreads, 0, s>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
@@ -695,7 +765,14 @@ cudaError_t launch_gemv_i8(const ifq_layer* Ls, int count, int T, void* ws, uint
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_i8_kernel, p);
+  return cudaLaunchKernelEx(&cfg, gemv_i8_kernel<P>, p);
+}
+
+}  // namespace
+
+cudaError_t launch_gemv_i8(const ifq_layer* Ls, int count, int T, void* ws, uint32_t* dev_status, cudaStream_t s) {
+  return count <= 8 ? launch_cap<8>(Ls, count, T, ws, dev_status, s)
+                    : launch_cap<IFQ_MAX_GROUP>(Ls, count, T, ws, dev_status, s);
 }
 
 }  // namespace ifq

@@ -2,6 +2,7 @@
 // files.  Arguments are validated by the caller; these only enqueue work.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -24,6 +25,12 @@ cudaError_t launch_gemv(const ifq_layer* L, int count, int T, int B, uint32_t* d
 // B = 1 integer tensor-core path (gemv_i8.cu) and its workspace size.
 size_t gemv_i8_workspace_bytes(const ifq_layer* L, int count, int T);
 cudaError_t launch_gemv_i8(const ifq_layer* L, int count, int T, void* ws, uint32_t* dev_status, cudaStream_t s);
+
+// Tiled TMA descriptor (cuTensorMapEncodeTiled through the runtime's driver entry point; no
+// libcuda link).  strides: rank - 1 byte strides of dimensions 1.. ; zero fill out of bounds.
+// False if the entry point is missing or the driver rejects the description.
+bool encode_tiled_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+                      const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle sw);
 
 cudaError_t launch_gemm(const ifq_layer* L, int count, int T, int64_t M, uint32_t* dev_status, cudaStream_t s);
 

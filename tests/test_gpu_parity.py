@@ -341,7 +341,7 @@ def _b1_case(rng, N, K, T, conj, xr32, xi32):
     return d, host, W.bf16_to_f32_numpy(xr), W.bf16_to_f32_numpy(xi), int(st.item())
 
 
-@pytest.mark.parametrize("K", [64, 192, 1024, 1088, 2048, 5504])
+@pytest.mark.parametrize("K", [64, 192, 1024, 1088, 2048, 3904, 5504])
 def test_b1_ragged_k_blocks(K):
     rng = np.random.default_rng(K)
     N, T = 77, 2
