@@ -163,6 +163,15 @@ class Block:
         self.gemv_ws = torch.zeros(max(16, Q.ifq_gemv_workspace_bytes(self.gemv_layers, self.T, self.B)),
                                    dtype=torch.uint8, device=dev)
         self.gemm_layers = self._layers(self.cfg4, self.M)
+        # the same conversion and quantization as one fused call per block (next-row measurement)
+        self.wl_layers = []
+        for i in range(len(self.cfg.layers)):
+            p = self.planes[i]
+            (cu, su), (cw, sw) = self.codes[2 * i], self.codes[2 * i + 1]
+            self.wl_layers.append(dict(R=self.R[i], U_re=p[0], U_im=p[1], W_re=p[2], W_im=p[3],
+                                       codes_u=cu, scales_u=su, codes_w=cw, scales_w=sw))
+        self.wl_ws = torch.empty(Q.ifq_widely_linear_quantize_workspace_bytes(self.wl_layers, self.T),
+                                 dtype=torch.uint8, device=dev)
 
     def _layers(self, cfg, rows):
         out = []
@@ -184,6 +193,13 @@ class Block:
         T = self.T
         per_entry = 8 * T + sum(t / 4 for t in range(T)) + T / 4
         return int(2 * sum(l.N * l.K for l in self.cfg.layers) * per_entry)
+
+    def fused_bytes(self):
+        # stage 1 fused with the conversion: R read (16 B), U and W written (16 B), two code bytes/4 written;
+        # stage t >= 2: U and W read (16 B), 2 (t-1)/4 earlier code bytes read, 2/4 written
+        T = self.T
+        per_pos = 32.5 + sum(16 + 0.5 * (t - 1) + 0.5 for t in range(2, T + 1))
+        return int(per_pos * sum(l.N * l.K for l in self.cfg.layers))
 
     def gemv_bytes(self, B):
         codes = W.code_bytes(self.cfg)
@@ -289,6 +305,28 @@ def decode_b16(block, reps=20):
 
 
 # ---------------------------------------------------------------- dense comparator
+def fused_convert_quantize(block, reps=10):
+    """Conversion fused with stage 1 of the quantizer (one call for the block's seven layers), timed
+    with CUDA events; its inputs (3.2 GB of R) are far larger than L2.  Reported beside the two-pass
+    conversion + quantizer times of the step, which compute the same outputs bit for bit."""
+    times = []
+    for k in range(reps + 3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        Q.ifq_widely_linear_quantize_pack(block.wl_layers, block.T, block.wl_ws, dev_status=block.status)
+        b.record()
+        torch.cuda.synchronize()
+        if k >= 3:
+            times.append(a.elapsed_time(b) * 1e-3)
+    assert int(block.status.item()) == 0, "device status set by the fused call"
+    t = statistics.median(times)
+    hbm = float(peaks()[0]["hbm_gbs"])
+    gbs = block.fused_bytes() / t / 1e9
+    return {"us": t * 1e6, "algorithmic_bytes": block.fused_bytes(), "GBps": gbs, "frac_of_hbm": gbs / hbm,
+            "launches": 1 + block.T - 1, "bytes_per_complex_position": block.fused_bytes() /
+            sum(l.N * l.K for l in block.cfg.layers)}
+
+
 def dense_comparator(block, reps=20):
     """Context, not the product: the original real layers of the block as dense bf16 matrices
     multiplied by cuBLAS (torch.matmul) -- decode at B = 1 with an L2 flush before every call,
@@ -441,6 +479,10 @@ def run_ours(args):
     if rank == 0 and ws == 1 and not args.skip_cpu_baseline:
         cpu = oracle_decode_sample(seconds_budget=args.cpu_seconds)
     b16 = decode_b16(block) if rank == 0 else None
+    fused = fused_convert_quantize(block) if rank == 0 else None
+    if fused is not None:
+        fused["two_pass_us"] = (t_conv + t_quant) * 1e6
+        fused["speedup_over_two_pass"] = (t_conv + t_quant) / (fused["us"] * 1e-6)
     if b16 is not None:
         b16["frac_of_hbm"] = b16["GBps"] / float(peaks()[0]["hbm_gbs"])
     dense = None
@@ -496,6 +538,7 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "decode_b16": b16,
+        "fused_convert_quantize": fused,
         "dense_bf16_comparator": dense,
         "gpu_launches": block.launches_per_step() * args.steps,
         "clocks": clk,
@@ -588,6 +631,20 @@ def run_case(args):
         def fn():
             Q.ifq_quantize_pack(ts, 2, wsb)
         label = "quantize c3 gate U+W T=2"
+    elif args.case == "wlq":
+        cfg = W.config("c3")
+        spec = cfg.layers[4]
+        R = 0.02 * torch.randn(spec.real_shape, device=dev, generator=g)
+        f = lambda: torch.empty((spec.N, spec.K), device=dev)  # noqa: E731
+        cb = lambda: torch.empty((2, spec.N, spec.K // 4), dtype=torch.uint8, device=dev)  # noqa: E731
+        wl = [dict(R=R, U_re=f(), U_im=f(), W_re=f(), W_im=f(), codes_u=cb(), scales_u=torch.empty((2, 2), device=dev),
+                   codes_w=cb(), scales_w=torch.empty((2, 2), device=dev))]
+        wsb = torch.empty(Q.ifq_widely_linear_quantize_workspace_bytes(wl, 2), dtype=torch.uint8, device=dev)
+        nbytes = 49.5 * spec.N * spec.K
+
+        def fn():
+            Q.ifq_widely_linear_quantize_pack(wl, 2, wsb)
+        label = "fused convert + quantize c3 gate T=2"
     elif args.case == "convert":
         cfg = W.config("c3")
         spec = cfg.layers[4]
@@ -625,7 +682,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--case", choices=["gemv", "gemm", "quant", "convert"], default=None)
+    ap.add_argument("--case", choices=["gemv", "gemm", "quant", "convert", "wlq"], default=None)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--workload", choices=["c3", "c5"], default="c5", help="layer set of --case gemv")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

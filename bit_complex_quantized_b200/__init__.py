@@ -23,5 +23,7 @@ from ._lib import (  # noqa: F401
     ifq_quantize_workspace_bytes,
     ifq_status_string,
     ifq_widely_linear_from_real,
+    ifq_widely_linear_quantize_pack,
+    ifq_widely_linear_quantize_workspace_bytes,
     load,
 )

@@ -26,6 +26,8 @@ EXPORTED = (
     "ifq_quantize_workspace_bytes",
     "ifq_quantize_pack",
     "ifq_quantize_pack_static",
+    "ifq_widely_linear_quantize_workspace_bytes",
+    "ifq_widely_linear_quantize_pack",
     "ifq_gemv_workspace_bytes",
     "ifq_gemv",
     "ifq_gemm",
@@ -47,6 +49,13 @@ class IfqError(RuntimeError):
 class QTensor(ctypes.Structure):
     _fields_ = [("w_re", ctypes.c_void_p), ("w_im", ctypes.c_void_p), ("N", ctypes.c_int64),
                 ("K", ctypes.c_int64), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+class WlLayer(ctypes.Structure):
+    _fields_ = [("R", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("U_re", ctypes.c_void_p), ("U_im", ctypes.c_void_p), ("W_re", ctypes.c_void_p),
+                ("W_im", ctypes.c_void_p), ("codes_u", ctypes.c_void_p), ("scales_u", ctypes.c_void_p),
+                ("codes_w", ctypes.c_void_p), ("scales_w", ctypes.c_void_p)]
 
 
 class Layer(ctypes.Structure):
@@ -78,6 +87,10 @@ def load():
     lib.ifq_quantize_pack.argtypes = [ctypes.POINTER(QTensor), i32, i32, vp, sz, vp, vp]
     lib.ifq_quantize_pack_static.restype = i32
     lib.ifq_quantize_pack_static.argtypes = [ctypes.POINTER(QTensor), i32, i32, vp, vp]
+    lib.ifq_widely_linear_quantize_workspace_bytes.restype = sz
+    lib.ifq_widely_linear_quantize_workspace_bytes.argtypes = [ctypes.POINTER(WlLayer), i32, i32]
+    lib.ifq_widely_linear_quantize_pack.restype = i32
+    lib.ifq_widely_linear_quantize_pack.argtypes = [ctypes.POINTER(WlLayer), i32, i32, vp, sz, vp, vp]
     lib.ifq_gemv_workspace_bytes.restype = sz
     lib.ifq_gemv_workspace_bytes.argtypes = [ctypes.POINTER(Layer), i32, i32, i32]
     lib.ifq_gemv.restype = i32
@@ -140,6 +153,30 @@ def ifq_quantize_pack_static(tensors, T, dev_status=None, stream=None):
     """As ifq_quantize_pack, with the library's fixed device scratch instead of a workspace."""
     arr = _qtensors(tensors)
     _check(load().ifq_quantize_pack_static(arr, len(tensors), T, _ptr(dev_status), _stream(stream)))
+
+
+def _wl_layers(layers):
+    arr = (WlLayer * len(layers))()
+    for i, d in enumerate(layers):
+        R = d["R"]
+        arr[i] = WlLayer(R.data_ptr(), R.shape[0], R.shape[1], _ptr(d["U_re"]), _ptr(d["U_im"]), _ptr(d["W_re"]),
+                         _ptr(d["W_im"]), _ptr(d["codes_u"]), _ptr(d["scales_u"]), _ptr(d["codes_w"]),
+                         _ptr(d["scales_w"]))
+    return arr
+
+
+def ifq_widely_linear_quantize_workspace_bytes(layers, T):
+    """layers: list of dicts with R [2n][2m] f32, U_re, U_im, W_re, W_im [n][m] f32,
+    codes_u, codes_w u8 [T][n][m/4], scales_u, scales_w f32 [T][2] (all on the device)."""
+    return int(load().ifq_widely_linear_quantize_workspace_bytes(_wl_layers(layers), len(layers), T))
+
+
+def ifq_widely_linear_quantize_pack(layers, T, workspace, dev_status=None, stream=None, workspace_bytes=None):
+    """Conversion and T-stage quantization of each layer in one call, stage 1 fused with the conversion."""
+    arr = _wl_layers(layers)
+    nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check(load().ifq_widely_linear_quantize_pack(arr, len(layers), T, _ptr(workspace), nbytes, _ptr(dev_status),
+                                                  _stream(stream)))
 
 
 def _layers(layers):

@@ -121,6 +121,45 @@ ifq_status ifq_quantize_pack_static(const ifq_qtensor* tensors, int count, int T
   return from_cuda(ifq::launch_quantize_static(tensors, count, T, dev_status, as_stream(stream)));
 }
 
+static ifq_status check_wl_layers(const ifq_wl_layer* layers, int count, int T) {
+  if (!layers) return IFQ_ERR_NULL;
+  if (count < 1 || count > IFQ_MAX_GROUP / 2) return IFQ_ERR_COUNT;
+  if (T < 1 || T > IFQ_MAX_STAGES) return IFQ_ERR_STAGES;
+  for (int i = 0; i < count; ++i) {
+    const ifq_wl_layer& l = layers[i];
+    if (!l.R || !l.U_re || !l.U_im || !l.W_re || !l.W_im || !l.codes_u || !l.scales_u || !l.codes_w || !l.scales_w)
+      return IFQ_ERR_NULL;
+    if (l.rows < 2 || (l.rows & 1) || l.cols < 8 || (l.cols % 8) != 0) return IFQ_ERR_SHAPE;
+    const int64_t n = l.rows / 2, m = l.cols / 2;
+    if (m > (int64_t)1 << 30 || n > ((int64_t)1 << 40) / m) return IFQ_ERR_SHAPE;
+    if (!aligned16(l.R) || !aligned16(l.U_re) || !aligned16(l.U_im) || !aligned16(l.W_re) || !aligned16(l.W_im) ||
+        !aligned16(l.codes_u) || !aligned16(l.codes_w) || (reinterpret_cast<uintptr_t>(l.scales_u) & 3u) ||
+        (reinterpret_cast<uintptr_t>(l.scales_w) & 3u))
+      return IFQ_ERR_ALIGN;
+  }
+  return IFQ_OK;
+}
+
+size_t ifq_widely_linear_quantize_workspace_bytes(const ifq_wl_layer* layers, int count, int T) {
+  if (!layers || count < 1 || count > IFQ_MAX_GROUP / 2) return 0;
+  (void)T;
+  for (int i = 0; i < count; ++i)
+    if (layers[i].rows < 2 || (layers[i].rows & 1) || layers[i].cols < 8 || (layers[i].cols % 8) != 0) return 0;
+  return ifq::widely_linear_quant_workspace_bytes(layers, count);
+}
+
+ifq_status ifq_widely_linear_quantize_pack(const ifq_wl_layer* layers, int count, int T, void* workspace,
+                                           size_t workspace_bytes, uint32_t* dev_status, ifq_stream_t stream) {
+  ifq_status st = check_wl_layers(layers, count, T);
+  if (st != IFQ_OK) return st;
+  if (!workspace || workspace_bytes < ifq::widely_linear_quant_workspace_bytes(layers, count))
+    return IFQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return IFQ_ERR_ALIGN;
+  st = check_device();
+  if (st != IFQ_OK) return st;
+  return from_cuda(ifq::launch_widely_linear_quantize(layers, count, T, workspace, dev_status, as_stream(stream)));
+}
+
 size_t ifq_gemv_workspace_bytes(const ifq_layer* layers, int count, int T, int B) {
   if (check_layers(layers, count, T) != IFQ_OK || B < 1 || B > IFQ_MAX_GEMV_BATCH) return 0;
   return B == 1 ? ifq::gemv_i8_workspace_bytes(layers, count, T) : 0;

@@ -20,6 +20,11 @@ cudaError_t launch_quantize(const ifq_qtensor* t, int count, int T, void* ws, ui
 // As launch_quantize, with the scratch in a file-scope device array (no allocation).
 cudaError_t launch_quantize_static(const ifq_qtensor* t, int count, int T, uint32_t* dev_status, cudaStream_t s);
 
+// Conversion fused with stage 1 of the quantizer, then stages 2..T (quantize.cu).
+size_t widely_linear_quant_workspace_bytes(const ifq_wl_layer* L, int count);
+cudaError_t launch_widely_linear_quantize(const ifq_wl_layer* L, int count, int T, void* ws, uint32_t* dev_status,
+                                          cudaStream_t s);
+
 cudaError_t launch_gemv(const ifq_layer* L, int count, int T, int B, uint32_t* dev_status, cudaStream_t s);
 
 // B = 1 integer tensor-core path (gemv_i8.cu) and its workspace size.

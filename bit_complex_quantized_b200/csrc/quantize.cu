@@ -259,6 +259,202 @@ void launch_stage(const QParams& p, unsigned blocks, cudaStream_t s) {
   quant_stage_kernel<PREV><<<blocks, kQThreads, 0, s>>>(p);
 }
 
+// ---------------------------------------------------------------- conversion fused with stage 1
+// ("Fairy2i write-up" §2.1 then §3.1, §3.2.)  One pass over R per layer: the
+// block computes U and W for its quads exactly as widely_linear_vec4_kernel
+// does, writes them (later stages read them), and runs stage 1 of both
+// tensors exactly as quant_stage_kernel<0> does -- same quads per thread, same
+// per-quad and per-block sums, same reduction order -- so codes, scales and
+// planes equal those of the two-pass path bit for bit.  HBM traffic per
+// complex position: 16 B of R read, 16 B of U, W and 0.5 B of codes written
+// (the two-pass path also reads U, W back: 48.5 B).
+struct FLayer {
+  const float* R;      // [2n][2m]
+  int64_t n, m;        // U, W are [n][m]
+  int64_t fblock_begin;
+  QTensorArg u, w;     // w_re / w_im of these are the planes this kernel writes
+};
+
+struct FParams {
+  FLayer L[IFQ_MAX_GROUP / 2];
+  int count;
+  uint32_t* status;
+};
+
+__device__ __forceinline__ float half_sum(float a, float b) { return __fmul_rn(0.5f, __fadd_rn(a, b)); }
+__device__ __forceinline__ float half_diff(float a, float b) { return __fmul_rn(0.5f, __fsub_rn(a, b)); }
+
+// Stage-1 results of one tensor's block: partial in slot blk, ticket taken by the caller.
+__device__ __forceinline__ void finish_scales(const QTensorArg& T) {
+  double a = 0.0, b = 0.0;
+  unsigned long long c = 0;
+  for (int64_t i = threadIdx.x; i < T.nblocks; i += kQThreads) {
+    const QPartial* pp = T.partials + i;
+    a += __ldcg(&pp->s_re);
+    b += __ldcg(&pp->s_im);
+    c += __ldcg(&pp->c_re);
+  }
+  block_sum3(a, b, c);
+  if (threadIdx.x == 0) {
+    const unsigned long long total = (unsigned long long)T.nquads * 4ull;
+    const unsigned long long c_im = total - c;
+    T.scales[0] = c > 0 ? (float)(a / (double)c) : 0.0f;
+    T.scales[1] = c_im > 0 ? (float)(b / (double)c_im) : 0.0f;
+  }
+}
+
+__global__ void __launch_bounds__(kQThreads) widely_linear_quant1_kernel(const __grid_constant__ FParams p) {
+  int li = 0;
+  while (li + 1 < p.count && (int64_t)blockIdx.x >= p.L[li + 1].fblock_begin) ++li;
+  const FLayer& L = p.L[li];
+  const int64_t blk = (int64_t)blockIdx.x - L.fblock_begin;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t quad0 = blk * kQuadsPerBlock + (int64_t)warp * (32 * kQuadsPerThread) + lane;
+  const int64_t m4 = L.m >> 2, half_row = L.m >> 1;  // float4s per output row; per R row = 2 m4
+  const int64_t nq = L.u.nquads;
+  const float4* R4 = reinterpret_cast<const float4*>(L.R);
+
+  // All loads first (16 x 128-bit per thread), then quad by quad: U and W, their
+  // stores, and stage-1 codes in the same quad order as quant_stage_kernel<0>.
+  float4 r11[kQuadsPerThread], r12[kQuadsPerThread], r21[kQuadsPerThread], r22[kQuadsPerThread];
+#pragma unroll
+  for (int q = 0; q < kQuadsPerThread; ++q) {
+    const int64_t quad = quad0 + 32 * q;
+    r11[q] = r12[q] = r21[q] = r22[q] = make_float4(0, 0, 0, 0);
+    if (quad < nq) {
+      // output row i, float4 column j4 of U / W (32-bit division when the operands fit)
+      const int64_t i = (quad | m4) < ((int64_t)1 << 32) ? (int64_t)((uint32_t)quad / (uint32_t)m4) : quad / m4;
+      const int64_t j4 = quad - i * m4;
+      const int64_t top = i * half_row + j4, bot = (i + L.n) * half_row + j4;
+      r11[q] = __ldcs(R4 + top);
+      r12[q] = __ldcs(R4 + top + m4);
+      r21[q] = __ldcs(R4 + bot);
+      r22[q] = __ldcs(R4 + bot + m4);
+    }
+  }
+
+  const uint32_t none[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  const double zero8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  double Su_re = 0.0, Su_im = 0.0, Sw_re = 0.0, Sw_im = 0.0;
+  unsigned long long Cu = 0, Cw = 0;
+  bool bad = false;
+#pragma unroll
+  for (int q = 0; q < kQuadsPerThread; ++q) {
+    const int64_t quad = quad0 + 32 * q;
+    if (quad >= nq) break;
+    const float a11[4] = {r11[q].x, r11[q].y, r11[q].z, r11[q].w}, a12[4] = {r12[q].x, r12[q].y, r12[q].z, r12[q].w};
+    const float a21[4] = {r21[q].x, r21[q].y, r21[q].z, r21[q].w}, a22[4] = {r22[q].x, r22[q].y, r22[q].z, r22[q].w};
+    float ur[4], ui[4], wr[4], wi[4];
+    float z = 0.0f;  // NaN iff some entry of this quad's U or W is NaN or infinite
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      ur[e] = half_sum(a11[e], a22[e]);
+      ui[e] = half_diff(a21[e], a12[e]);
+      wr[e] = half_diff(a11[e], a22[e]);
+      wi[e] = half_sum(a12[e], a21[e]);
+      z += (ur[e] * 0.0f + ui[e] * 0.0f) + (wr[e] * 0.0f + wi[e] * 0.0f);
+    }
+    reinterpret_cast<float4*>(const_cast<float*>(L.u.w_re))[quad] = make_float4(ur[0], ur[1], ur[2], ur[3]);
+    reinterpret_cast<float4*>(const_cast<float*>(L.u.w_im))[quad] = make_float4(ui[0], ui[1], ui[2], ui[3]);
+    reinterpret_cast<float4*>(const_cast<float*>(L.w.w_re))[quad] = make_float4(wr[0], wr[1], wr[2], wr[3]);
+    reinterpret_cast<float4*>(const_cast<float*>(L.w.w_im))[quad] = make_float4(wi[0], wi[1], wi[2], wi[3]);
+    // The checked form differs from the plain one only on non-finite entries.
+    const bool bq = z != 0.0f;
+    bad |= bq;
+    const uint32_t bu = bq ? quad_code<0, true>(ur, ui, none, zero8, zero8, Su_re, Su_im)
+                           : quad_code<0, false>(ur, ui, none, zero8, zero8, Su_re, Su_im);
+    const uint32_t bw = bq ? quad_code<0, true>(wr, wi, none, zero8, zero8, Sw_re, Sw_im)
+                           : quad_code<0, false>(wr, wi, none, zero8, zero8, Sw_re, Sw_im);
+    Cu += 4u - (uint32_t)__popc(bu & 0x55u);
+    Cw += 4u - (uint32_t)__popc(bw & 0x55u);
+    L.u.codes[quad] = (uint8_t)bu;
+    L.w.codes[quad] = (uint8_t)bw;
+  }
+  if (__syncthreads_or(bad) && threadIdx.x == 0) set_status(p.status, IFQ_DEV_NONFINITE);
+
+  block_sum3(Su_re, Su_im, Cu);
+  block_sum3(Sw_re, Sw_im, Cw);
+  __shared__ int am_last;
+  if (threadIdx.x == 0) {
+    QPartial pu, pw;
+    pu.s_re = Su_re;
+    pu.s_im = Su_im;
+    pu.c_re = Cu;
+    pu.pad = 0;
+    pw.s_re = Sw_re;
+    pw.s_im = Sw_im;
+    pw.c_re = Cw;
+    pw.pad = 0;
+    L.u.partials[blk] = pu;
+    L.w.partials[blk] = pw;
+    __threadfence();
+    const unsigned prev_ticket = atomicAdd(L.u.ticket, 1u);  // one ticket counts the layer's blocks
+    am_last = (prev_ticket == (unsigned)(L.u.nblocks - 1));
+  }
+  __syncthreads();
+  if (!am_last) return;
+  __threadfence();
+  finish_scales(L.u);
+  finish_scales(L.w);
+  if (threadIdx.x == 0) *L.u.ticket = 0u;  // re-armed for the stage launches that follow
+}
+
+// Fills p for `count` tensors over the workspace (tickets, then partials) and
+// returns the total number of blocks of one stage launch.
+int64_t fill_qparams(const ifq_qtensor* t, int count, void* ws, QParams& p, size_t* ticket_bytes) {
+  memset(&p, 0, sizeof(p));
+  p.count = count;
+  char* base = static_cast<char*>(ws);
+  *ticket_bytes = ((size_t)count * 16 + 255) / 256 * 256;
+  char* part = base + *ticket_bytes;
+  int64_t blocks = 0;
+  for (int i = 0; i < count; ++i) {
+    QTensorArg& a = p.t[i];
+    a.w_re = t[i].w_re;
+    a.w_im = t[i].w_im;
+    a.codes = t[i].codes;
+    a.scales = t[i].scales;
+    a.nquads = t[i].N * t[i].K / 4;
+    a.nblocks = quant_blocks_for(t[i].N, t[i].K);
+    a.block_begin = blocks;
+    a.ticket = reinterpret_cast<unsigned int*>(base + 16 * i);
+    a.partials = reinterpret_cast<QPartial*>(part);
+    part += (size_t)a.nblocks * sizeof(QPartial);
+    blocks += a.nblocks;
+  }
+  return blocks;
+}
+
+// Stage launches st_begin .. T-1 over every tensor of p.
+cudaError_t launch_stages(QParams& p, int64_t blocks, int st_begin, int T, cudaStream_t s) {
+  for (int st = st_begin; st < T; ++st) {
+    p.stage = st;
+    const unsigned nb = (unsigned)blocks;
+    switch (st) {
+      case 0: launch_stage<0>(p, nb, s); break;
+      case 1: launch_stage<1>(p, nb, s); break;
+      case 2: launch_stage<2>(p, nb, s); break;
+      case 3: launch_stage<3>(p, nb, s); break;
+      case 4: launch_stage<4>(p, nb, s); break;
+      case 5: launch_stage<5>(p, nb, s); break;
+      case 6: launch_stage<6>(p, nb, s); break;
+      default: launch_stage<7>(p, nb, s); break;
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+// The 2 count tensors (U_0, W_0, U_1, W_1, ...) of a fused call.
+void fused_tensors(const ifq_wl_layer* Ls, int count, ifq_qtensor* t) {
+  for (int i = 0; i < count; ++i) {
+    const int64_t n = Ls[i].rows / 2, m = Ls[i].cols / 2;
+    t[2 * i] = ifq_qtensor{Ls[i].U_re, Ls[i].U_im, n, m, Ls[i].codes_u, Ls[i].scales_u};
+    t[2 * i + 1] = ifq_qtensor{Ls[i].W_re, Ls[i].W_im, n, m, Ls[i].codes_w, Ls[i].scales_w};
+  }
+}
+
 }  // namespace
 
 int64_t quant_blocks_for(int64_t N, int64_t K) {
@@ -275,47 +471,51 @@ size_t quant_workspace_bytes(const ifq_qtensor* t, int count) {
 
 cudaError_t launch_quantize(const ifq_qtensor* t, int count, int T, void* ws, uint32_t* dev_status, cudaStream_t s) {
   QParams p;
-  memset(&p, 0, sizeof(p));
-  p.count = count;
+  size_t ticket_bytes = 0;
+  const int64_t blocks = fill_qparams(t, count, ws, p, &ticket_bytes);
   p.status = dev_status;
-  char* base = static_cast<char*>(ws);
-  const size_t ticket_bytes = ((size_t)count * 16 + 255) / 256 * 256;
-  char* part = base + ticket_bytes;
-  int64_t blocks = 0;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  cudaError_t e = cudaMemsetAsync(ws, 0, ticket_bytes, s);
+  if (e != cudaSuccess) return e;
+  return launch_stages(p, blocks, 0, T, s);
+}
+
+size_t widely_linear_quant_workspace_bytes(const ifq_wl_layer* Ls, int count) {
+  ifq_qtensor t[IFQ_MAX_GROUP];
+  fused_tensors(Ls, count, t);
+  return quant_workspace_bytes(t, 2 * count);
+}
+
+cudaError_t launch_widely_linear_quantize(const ifq_wl_layer* Ls, int count, int T, void* ws, uint32_t* dev_status,
+                                          cudaStream_t s) {
+  ifq_qtensor t[IFQ_MAX_GROUP];
+  fused_tensors(Ls, count, t);
+  QParams p;
+  size_t ticket_bytes = 0;
+  const int64_t blocks = fill_qparams(t, 2 * count, ws, p, &ticket_bytes);
+  p.status = dev_status;
+  FParams f;
+  memset(&f, 0, sizeof(f));
+  f.count = count;
+  f.status = dev_status;
+  int64_t fblocks = 0;
   for (int i = 0; i < count; ++i) {
-    QTensorArg& a = p.t[i];
-    a.w_re = t[i].w_re;
-    a.w_im = t[i].w_im;
-    a.codes = t[i].codes;
-    a.scales = t[i].scales;
-    a.nquads = t[i].N * t[i].K / 4;
-    a.nblocks = quant_blocks_for(t[i].N, t[i].K);
-    a.block_begin = blocks;
-    a.ticket = reinterpret_cast<unsigned int*>(base + 16 * i);
-    a.partials = reinterpret_cast<QPartial*>(part);
-    part += (size_t)a.nblocks * sizeof(QPartial);
-    blocks += a.nblocks;
+    FLayer& a = f.L[i];
+    a.R = Ls[i].R;
+    a.n = Ls[i].rows / 2;
+    a.m = Ls[i].cols / 2;
+    a.fblock_begin = fblocks;
+    a.u = p.t[2 * i];
+    a.w = p.t[2 * i + 1];
+    fblocks += a.u.nblocks;
   }
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaMemsetAsync(base, 0, ticket_bytes, s);
+  cudaError_t e = cudaMemsetAsync(ws, 0, ticket_bytes, s);
   if (e != cudaSuccess) return e;
-  for (int st = 0; st < T; ++st) {
-    p.stage = st;
-    const unsigned nb = (unsigned)blocks;
-    switch (st) {
-      case 0: launch_stage<0>(p, nb, s); break;
-      case 1: launch_stage<1>(p, nb, s); break;
-      case 2: launch_stage<2>(p, nb, s); break;
-      case 3: launch_stage<3>(p, nb, s); break;
-      case 4: launch_stage<4>(p, nb, s); break;
-      case 5: launch_stage<5>(p, nb, s); break;
-      case 6: launch_stage<6>(p, nb, s); break;
-      default: launch_stage<7>(p, nb, s); break;
-    }
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  return cudaSuccess;
+  widely_linear_quant1_kernel<<<(unsigned)fblocks, kQThreads, 0, s>>>(f);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_stages(p, blocks, 1, T, s);
 }
 
 // Scratch of ifq_quantize_pack_static, for callers that cannot hand over device

@@ -162,6 +162,54 @@ ifq_status ifq_quantize_pack_static(const ifq_qtensor* tensors, int count, int T
                                     ifq_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * ifq_widely_linear_quantize_pack  ("Fairy2i write-up" §2.1, then §3.1, §3.2, §4.1)
+ *
+ * ifq_widely_linear_from_real followed by ifq_quantize_pack of the resulting
+ * U and W, with the conversion and stage 1 done in one pass over R: every
+ * output -- the four planes, the codes and the scales of every stage -- is
+ * bit for bit what the two calls give.  Per complex position at stage 1 this
+ * moves 32.5 bytes of HBM traffic instead of 48.5 (R is read once; U and W are
+ * written and not read back until stage 2).  Stages 2..T run as in
+ * ifq_quantize_pack.
+ *
+ *   layers[i].R                  [rows][cols] float32, device, read-only
+ *   layers[i].rows, cols         rows even >= 2; cols >= 8, cols % 8 == 0
+ *                                (U, W are n x m = rows/2 x cols/2, m % 4 == 0)
+ *   layers[i].U_re .. W_im       [n][m] float32, device, written (the
+ *                                conversion's output and the quantizer's input)
+ *   layers[i].codes_u, codes_w   [T][n][m/4] uint8, device, written
+ *   layers[i].scales_u, scales_w [T][2] float32, device, written
+ *   count                        1..IFQ_MAX_GROUP/2 layers (U and W count as
+ *                                two tensors of one ifq_quantize_pack call)
+ *   T                            1..IFQ_MAX_STAGES
+ *   workspace                    device scratch of
+ *                                ifq_widely_linear_quantize_workspace_bytes()
+ *                                bytes, 16-byte aligned, owned by the caller;
+ *                                no initial contents needed
+ *   dev_status                   device uint32, bits OR-ed in (may be NULL)
+ * Pointers must be 16-byte aligned (scales: 4-byte).  No output may overlap R
+ * or another output.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  const float* R;
+  int64_t rows;
+  int64_t cols;
+  float* U_re;
+  float* U_im;
+  float* W_re;
+  float* W_im;
+  uint8_t* codes_u;
+  float* scales_u;
+  uint8_t* codes_w;
+  float* scales_w;
+} ifq_wl_layer;
+
+size_t ifq_widely_linear_quantize_workspace_bytes(const ifq_wl_layer* layers, int count, int T);
+
+ifq_status ifq_widely_linear_quantize_pack(const ifq_wl_layer* layers, int count, int T, void* workspace,
+                                           size_t workspace_bytes, uint32_t* dev_status, ifq_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Product layers ("Fairy2i write-up" §2.1, §4.2; "iFairy article" §二.2)
  *
  *   y = sum_t ( U_hat_t x + W_hat_t conj(x) ),  per token,

@@ -137,3 +137,34 @@ def test_layerset_marshals_the_same_descriptors():
     for x, y in zip(a, b.array):
         for f, _ in L.Layer._fields_:
             assert getattr(x, f) == getattr(y, f)
+
+
+def _wl(**kw):
+    d = dict(R=FAKE, rows=8, cols=16, U_re=FAKE, U_im=FAKE, W_re=FAKE, W_im=FAKE, codes_u=FAKE, scales_u=FAKE,
+             codes_w=FAKE, scales_w=FAKE)
+    d.update(kw)
+    return L.WlLayer(d["R"], d["rows"], d["cols"], d["U_re"], d["U_im"], d["W_re"], d["W_im"], d["codes_u"],
+                     d["scales_u"], d["codes_w"], d["scales_w"])
+
+
+def test_fused_convert_quantize_argument_errors():
+    lib = Q.load()
+    arr = (L.WlLayer * 1)(_wl())
+    need = lib.ifq_widely_linear_quantize_workspace_bytes(arr, 1, 2)
+    # same workspace as a quantizer call on the two 4 x 8 tensors U and W
+    qt = (L.QTensor * 2)(L.QTensor(FAKE, FAKE, 4, 8, FAKE, FAKE), L.QTensor(FAKE, FAKE, 4, 8, FAKE, FAKE))
+    assert need == lib.ifq_quantize_workspace_bytes(qt, 2, 2) > 0
+    call = lambda a, n=1, T=2, ws=FAKE, nb=need: lib.ifq_widely_linear_quantize_pack(a, n, T, ws, nb, None, None)
+    assert call(None) == 1
+    assert call(arr, n=0) == 9
+    assert call((L.WlLayer * 17)(*([_wl()] * 17)), n=17) == 9   # U and W count twice: at most 16 layers
+    assert call(arr, T=0) == 4 and call(arr, T=9) == 4
+    assert call((L.WlLayer * 1)(_wl(codes_w=None))) == 1
+    assert call((L.WlLayer * 1)(_wl(rows=7))) == 2
+    assert call((L.WlLayer * 1)(_wl(cols=12))) == 2            # m = 6 is not a multiple of 4
+    assert call((L.WlLayer * 1)(_wl(cols=4))) == 2
+    assert call((L.WlLayer * 1)(_wl(U_im=FAKE + 4))) == 3
+    assert call((L.WlLayer * 1)(_wl(scales_w=FAKE + 2))) == 3
+    assert call(arr, ws=None) == 6 and call(arr, nb=need - 1) == 6
+    assert call(arr, ws=FAKE + 8) == 3
+    assert lib.ifq_widely_linear_quantize_workspace_bytes((L.WlLayer * 1)(_wl(cols=12)), 1, 2) == 0
