@@ -4,7 +4,7 @@ Default run (the contract line): one step is one pass of the whole path on the
 LLaMA-2-7B-shaped Fairy2i block (seven real layers q,k,v,o 4096x4096,
 gate,up 4096->11008, down 11008->4096; 2 residual stages; U and W):
   1. widely-linear conversion of the seven real layers        (7 launches)
-  2. 2-stage PhaseQuant + pack of the 14 complex tensors      (1 memset + 2 launches)
+  2. 2-stage PhaseQuant + pack of the 14 complex tensors      (2 stage + 2 reduction launches)
   3. L2 flush (256 MiB memset), then decode GEMV at B = 1     (1 launch, all 7 layers)
   4. prefill GEMM at M = 2048 tokens                          (7 launches)
 Inputs are resident in HBM when the timed region starts; the metric value is
@@ -230,9 +230,10 @@ class Block:
             ev[5].record(s)
 
     def launches_per_step(self):
-        """Our kernels per step (the memsets are not counted): conversion, quantizer, GEMV, GEMM."""
+        """Our kernels per step (the L2-flush memset is not counted): conversion, quantizer (a stage
+        kernel and a reduction kernel per stage), GEMV, GEMM."""
         gemv = 2 if self.B == 1 else 1  # B = 1: activation prep + integer product
-        return len(self.cfg.layers) + 2 + gemv + len(self.gemm_layers)
+        return len(self.cfg.layers) + 2 * self.T + gemv + len(self.gemm_layers)
 
 
 def oracle_sample_layers(rows_per_layer):
@@ -323,7 +324,7 @@ def fused_convert_quantize(block, reps=10):
     hbm = float(peaks()[0]["hbm_gbs"])
     gbs = block.fused_bytes() / t / 1e9
     return {"us": t * 1e6, "algorithmic_bytes": block.fused_bytes(), "GBps": gbs, "frac_of_hbm": gbs / hbm,
-            "launches": 1 + block.T - 1, "bytes_per_complex_position": block.fused_bytes() /
+            "launches": 2 * block.T, "bytes_per_complex_position": block.fused_bytes() /
             sum(l.N * l.K for l in block.cfg.layers)}
 
 

@@ -1,22 +1,25 @@
 // PhaseQuant with axis scales and recursive residual stages
 // ("Fairy2i write-up" §3.1, §3.2, §4.1).
 //
-// One launch per stage t covers every tensor of the call.  Each thread takes
-// four quads (4 consecutive weights = one code byte) strided by 32 within its
-// warp, so every load and store instruction of a warp is contiguous:
-//   1. residual r_t = w - sum_{u<t} w_hat_u, rebuilt in float64 from w and the
-//      already written codes and float32 scales of the earlier stages (w is
+// Work unit: a tile of 1024 quads (4 consecutive weights = one code byte) of
+// one tensor.  Each thread of a 256-thread block takes four quads of the tile,
+// strided by 32 within its warp, and per stage t:
+//   1. rebuilds the residual r_t = w - sum_{u<t} w_hat_u in float64 from w and
+//      the already written codes and float32 scales of the earlier stages (w is
 //      read again each stage: the per-tensor scale of stage t-1 is a global
 //      dependency, and the fp32 weights of a layer do not fit on chip);
-//   2. the sector k of r_t by exact comparisons (no atan2);
-//   3. four codes packed into one byte;
-//   4. per-class sums S_re = sum |Re r| over k even, S_im = sum |Im r| over k
-//      odd and the class-0 count, in float64 / integer, reduced per block in a
-//      fixed order into workspace partials.
-// The last block of a tensor to finish (atomic ticket) reduces the partials in
-// block order and writes s_re = S_re/C_re, s_im = S_im/C_im (0 for an empty
-// class) rounded to float32, then re-arms the ticket for the next stage.
-// No block waits on another, so nothing can hang.
+//   2. finds the sector k of r_t by exact comparisons (no atan2);
+//   3. packs four codes into one byte;
+//   4. sums S_re = sum |Re r| over k even, S_im = sum |Im r| over k odd and the
+//      class-0 count (float64 / integer); the block reduces them in a fixed
+//      order into the tile's partial in the workspace.
+// A stage is two launches: quant_stage_kernel (one block per tile) and
+// quant_reduce_kernel (one block per tensor: the partials in tile order ->
+// s_re = S_re/C_re, s_im = S_im/C_im, 0 for an empty class, rounded to
+// float32).  Consecutive launches are chained with programmatic dependent
+// launch: a stage kernel loads its weights while the previous reduction runs
+// and waits for it only before it needs the earlier scales and codes.  No
+// block waits on another block of its own grid.
 #include "ifq_common.cuh"
 #include "ifq_internal.h"
 
@@ -27,7 +30,7 @@ namespace {
 
 constexpr int kQThreads = 256;
 constexpr int kQuadsPerThread = 4;
-constexpr int kQuadsPerBlock = kQThreads * kQuadsPerThread;
+constexpr int kQuadsPerBlock = kQThreads * kQuadsPerThread;  // one tile
 
 struct QPartial {
   double s_re;
@@ -41,19 +44,22 @@ struct QTensorArg {
   const float* w_im;
   uint8_t* codes;        // [T][nquads]
   float* scales;         // [T][2]
-  QPartial* partials;    // [nblocks]
-  unsigned int* ticket;  // one counter
+  QPartial* partials;    // [nblocks]: one per tile
   int64_t nquads;        // N*K/4
-  int64_t block_begin;   // first global block of this tensor
-  int64_t nblocks;
+  int64_t block_begin;   // first global tile of this tensor
+  int64_t nblocks;       // tiles
 };
 
 struct QParams {
   QTensorArg t[IFQ_MAX_GROUP];
+  int64_t tiles;  // tiles of all tensors (tensor-major)
   int count;
-  int stage;  // 0-based stage being computed
+  int stage;      // 0-based stage being computed
   uint32_t* status;
 };
+
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // Sector of w = a + ib as (cls, sgn) with k = 2 sgn + cls: 0 -> 1, 1 -> i,
 // 2 -> -1, 3 -> -i.  Written without branches for finite a, b in any IEEE
@@ -71,13 +77,6 @@ __device__ __forceinline__ uint32_t sector_code(F a, F b) {
   const uint32_t cls = (ab > aa) || tie_same;
   const uint32_t sgn = cls ? (b < F(0)) : (a < F(0));
   return 2u * sgn + cls;
-}
-
-// Exact reference form of the same rule, used for entries with a non-finite part
-// (taken as 0) on the rare slow path.
-__device__ __forceinline__ uint32_t sector_code_checked(float a, float b) {
-  if (!(isfinite(a) && isfinite(b))) return 0u;
-  return sector_code(a, b);
 }
 
 __device__ __forceinline__ double warp_sum(double v) {
@@ -162,8 +161,11 @@ __device__ __forceinline__ uint32_t quad_code(const float (&wr)[4], const float 
   return byte;
 }
 
+// ---------------------------------------------------------------- stage kernel
+// One block per tile; the block's partial goes to the tile's workspace slot.
 template <int PREV>
 __global__ void __launch_bounds__(kQThreads) quant_stage_kernel(const __grid_constant__ QParams p) {
+  pdl_trigger();  // the reduction of this stage may launch and wait for this grid
   // Find this block's tensor (at most IFQ_MAX_GROUP entries, uniform per block).
   int ti = 0;
   while (ti + 1 < p.count && (int64_t)blockIdx.x >= p.t[ti + 1].block_begin) ++ti;
@@ -172,16 +174,9 @@ __global__ void __launch_bounds__(kQThreads) quant_stage_kernel(const __grid_con
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t quad0 = blk * kQuadsPerBlock + (int64_t)warp * (32 * kQuadsPerThread) + lane;
 
-  double sr[8], si[8];
-#pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    sr[u] = u < PREV ? (double)__ldg(T.scales + 2 * u) : 0.0;
-    si[u] = u < PREV ? (double)__ldg(T.scales + 2 * u + 1) : 0.0;
-  }
-
-  // Load all four quads first (8 x 128-bit weight loads, PREV byte loads each).
+  // The weights are inputs of the call, never written by its earlier launches: their
+  // loads (8 x 128 bits per thread) go out before waiting for the previous launch.
   float wr[kQuadsPerThread][4], wi[kQuadsPerThread][4];
-  uint32_t prev[kQuadsPerThread][8];
 #pragma unroll
   for (int q = 0; q < kQuadsPerThread; ++q) {
     const int64_t quad = quad0 + 32 * q;
@@ -190,8 +185,21 @@ __global__ void __launch_bounds__(kQThreads) quant_stage_kernel(const __grid_con
     const float4 vi = ok ? __ldcs(reinterpret_cast<const float4*>(T.w_im) + quad) : make_float4(0, 0, 0, 0);
     wr[q][0] = vr.x; wr[q][1] = vr.y; wr[q][2] = vr.z; wr[q][3] = vr.w;
     wi[q][0] = vi.x; wi[q][1] = vi.y; wi[q][2] = vi.z; wi[q][3] = vi.w;
+  }
+  pdl_wait();  // the earlier stages' codes and scales are complete from here on
+  double sr[8], si[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) prev[q][u] = (u < PREV && ok) ? __ldg(T.codes + (int64_t)u * T.nquads + quad) : 0u;
+  for (int u = 0; u < 8; ++u) {
+    sr[u] = u < PREV ? (double)__ldg(T.scales + 2 * u) : 0.0;
+    si[u] = u < PREV ? (double)__ldg(T.scales + 2 * u + 1) : 0.0;
+  }
+  uint32_t prev[kQuadsPerThread][8];
+#pragma unroll
+  for (int q = 0; q < kQuadsPerThread; ++q) {
+    const int64_t quad = quad0 + 32 * q;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      prev[q][u] = (u < PREV && quad < T.nquads) ? __ldg(T.codes + (int64_t)u * T.nquads + quad) : 0u;
   }
 
   // Non-finite weights are rare: one check for all 16 entries, exact handling only then.
@@ -217,7 +225,6 @@ __global__ void __launch_bounds__(kQThreads) quant_stage_kernel(const __grid_con
   if (__syncthreads_or(bad) && threadIdx.x == 0) set_status(p.status, IFQ_DEV_NONFINITE);
 
   block_sum3(S_re, S_im, C_re);
-  __shared__ int am_last;
   if (threadIdx.x == 0) {
     QPartial part;
     part.s_re = S_re;
@@ -225,49 +232,42 @@ __global__ void __launch_bounds__(kQThreads) quant_stage_kernel(const __grid_con
     part.c_re = C_re;
     part.pad = 0;
     T.partials[blk] = part;
-    __threadfence();
-    const unsigned prev_ticket = atomicAdd(T.ticket, 1u);
-    am_last = (prev_ticket == (unsigned)(T.nblocks - 1));
   }
-  __syncthreads();
-  if (!am_last) return;
+}
 
-  // Last block of this tensor: reduce all partials in a fixed order.
-  __threadfence();
+// ---------------------------------------------------------------- scale reduction
+// One block per tensor: thread i adds the partials of tiles i, i + 256, ... in
+// order, then the block adds the threads' sums in a fixed tree.
+__global__ void __launch_bounds__(kQThreads) quant_reduce_kernel(const __grid_constant__ QParams p) {
+  pdl_trigger();  // the next stage may launch and start streaming its weights
+  pdl_wait();     // every tile partial of this stage is written
+  const QTensorArg& T = p.t[blockIdx.x];
   double a = 0.0, b = 0.0;
   unsigned long long c = 0;
   for (int64_t i = threadIdx.x; i < T.nblocks; i += kQThreads) {
     const QPartial* pp = T.partials + i;
-    a += __ldcg(&pp->s_re);
-    b += __ldcg(&pp->s_im);
-    c += __ldcg(&pp->c_re);
+    a += pp->s_re;
+    b += pp->s_im;
+    c += pp->c_re;
   }
   block_sum3(a, b, c);
   if (threadIdx.x == 0) {
     const unsigned long long total = (unsigned long long)T.nquads * 4ull;
     const unsigned long long c_im = total - c;
-    const float s_re = c > 0 ? (float)(a / (double)c) : 0.0f;
-    const float s_im = c_im > 0 ? (float)(b / (double)c_im) : 0.0f;
-    T.scales[2 * PREV] = s_re;
-    T.scales[2 * PREV + 1] = s_im;
-    *T.ticket = 0u;  // re-arm for the next stage launch
+    T.scales[2 * p.stage] = c > 0 ? (float)(a / (double)c) : 0.0f;
+    T.scales[2 * p.stage + 1] = c_im > 0 ? (float)(b / (double)c_im) : 0.0f;
   }
-}
-
-template <int PREV>
-void launch_stage(const QParams& p, unsigned blocks, cudaStream_t s) {
-  quant_stage_kernel<PREV><<<blocks, kQThreads, 0, s>>>(p);
 }
 
 // ---------------------------------------------------------------- conversion fused with stage 1
 // ("Fairy2i write-up" §2.1 then §3.1, §3.2.)  One pass over R per layer: the
 // block computes U and W for its quads exactly as widely_linear_vec4_kernel
 // does, writes them (later stages read them), and runs stage 1 of both
-// tensors exactly as quant_stage_kernel<0> does -- same quads per thread, same
-// per-quad and per-block sums, same reduction order -- so codes, scales and
-// planes equal those of the two-pass path bit for bit.  HBM traffic per
-// complex position: 16 B of R read, 16 B of U, W and 0.5 B of codes written
-// (the two-pass path also reads U, W back: 48.5 B).
+// tensors exactly as quant_stage_kernel<0> does -- same quads per thread,
+// same per-quad sums, same tile partials, then the same reduction kernel -- so
+// codes, scales and planes equal those of the two-pass path bit for bit.  HBM
+// traffic per complex position: 16 B of R read, 16 B of U, W and 0.5 B of
+// codes written (the two-pass path also reads U, W back: 48.5 B).
 struct FLayer {
   const float* R;      // [2n][2m]
   int64_t n, m;        // U, W are [n][m]
@@ -283,25 +283,6 @@ struct FParams {
 
 __device__ __forceinline__ float half_sum(float a, float b) { return __fmul_rn(0.5f, __fadd_rn(a, b)); }
 __device__ __forceinline__ float half_diff(float a, float b) { return __fmul_rn(0.5f, __fsub_rn(a, b)); }
-
-// Stage-1 results of one tensor's block: partial in slot blk, ticket taken by the caller.
-__device__ __forceinline__ void finish_scales(const QTensorArg& T) {
-  double a = 0.0, b = 0.0;
-  unsigned long long c = 0;
-  for (int64_t i = threadIdx.x; i < T.nblocks; i += kQThreads) {
-    const QPartial* pp = T.partials + i;
-    a += __ldcg(&pp->s_re);
-    b += __ldcg(&pp->s_im);
-    c += __ldcg(&pp->c_re);
-  }
-  block_sum3(a, b, c);
-  if (threadIdx.x == 0) {
-    const unsigned long long total = (unsigned long long)T.nquads * 4ull;
-    const unsigned long long c_im = total - c;
-    T.scales[0] = c > 0 ? (float)(a / (double)c) : 0.0f;
-    T.scales[1] = c_im > 0 ? (float)(b / (double)c_im) : 0.0f;
-  }
-}
 
 __global__ void __launch_bounds__(kQThreads) widely_linear_quant1_kernel(const __grid_constant__ FParams p) {
   int li = 0;
@@ -374,7 +355,6 @@ __global__ void __launch_bounds__(kQThreads) widely_linear_quant1_kernel(const _
 
   block_sum3(Su_re, Su_im, Cu);
   block_sum3(Sw_re, Sw_im, Cw);
-  __shared__ int am_last;
   if (threadIdx.x == 0) {
     QPartial pu, pw;
     pu.s_re = Su_re;
@@ -387,27 +367,16 @@ __global__ void __launch_bounds__(kQThreads) widely_linear_quant1_kernel(const _
     pw.pad = 0;
     L.u.partials[blk] = pu;
     L.w.partials[blk] = pw;
-    __threadfence();
-    const unsigned prev_ticket = atomicAdd(L.u.ticket, 1u);  // one ticket counts the layer's blocks
-    am_last = (prev_ticket == (unsigned)(L.u.nblocks - 1));
   }
-  __syncthreads();
-  if (!am_last) return;
-  __threadfence();
-  finish_scales(L.u);
-  finish_scales(L.w);
-  if (threadIdx.x == 0) *L.u.ticket = 0u;  // re-armed for the stage launches that follow
 }
 
-// Fills p for `count` tensors over the workspace (tickets, then partials) and
-// returns the total number of blocks of one stage launch.
-int64_t fill_qparams(const ifq_qtensor* t, int count, void* ws, QParams& p, size_t* ticket_bytes) {
+// Fills p for `count` tensors over the workspace (the tile partials) and
+// returns the number of tiles of one stage.
+int64_t fill_qparams(const ifq_qtensor* t, int count, void* ws, QParams& p) {
   memset(&p, 0, sizeof(p));
   p.count = count;
-  char* base = static_cast<char*>(ws);
-  *ticket_bytes = ((size_t)count * 16 + 255) / 256 * 256;
-  char* part = base + *ticket_bytes;
-  int64_t blocks = 0;
+  char* part = static_cast<char*>(ws);
+  int64_t tiles = 0;
   for (int i = 0; i < count; ++i) {
     QTensorArg& a = p.t[i];
     a.w_re = t[i].w_re;
@@ -416,31 +385,57 @@ int64_t fill_qparams(const ifq_qtensor* t, int count, void* ws, QParams& p, size
     a.scales = t[i].scales;
     a.nquads = t[i].N * t[i].K / 4;
     a.nblocks = quant_blocks_for(t[i].N, t[i].K);
-    a.block_begin = blocks;
-    a.ticket = reinterpret_cast<unsigned int*>(base + 16 * i);
+    a.block_begin = tiles;
     a.partials = reinterpret_cast<QPartial*>(part);
     part += (size_t)a.nblocks * sizeof(QPartial);
-    blocks += a.nblocks;
+    tiles += a.nblocks;
   }
-  return blocks;
+  p.tiles = tiles;
+  return tiles;
 }
 
-// Stage launches st_begin .. T-1 over every tensor of p.
-cudaError_t launch_stages(QParams& p, int64_t blocks, int st_begin, int T, cudaStream_t s) {
+// Launch with programmatic stream serialization (the kernel's pdl_wait orders
+// it after the previous launch) or, for the first launch of a call, plainly.
+template <class Kern>
+cudaError_t launch(Kern kern, unsigned grid, int smem, bool chained, const QParams& p, cudaStream_t s) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kQThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = chained ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+template <int PREV>
+cudaError_t launch_stage(const QParams& p, bool chained, cudaStream_t s) {
+  return launch(quant_stage_kernel<PREV>, (unsigned)p.tiles, 0, chained, p, s);
+}
+
+// Stages st_begin .. T-1 over every tensor of p: a stage kernel and its reduction each.
+// chained: the first stage kernel follows a launch of this call (not the caller's work).
+cudaError_t launch_stages(QParams& p, int st_begin, int T, bool chained, cudaStream_t s) {
   for (int st = st_begin; st < T; ++st) {
     p.stage = st;
-    const unsigned nb = (unsigned)blocks;
+    const bool ch = chained || st > st_begin;
+    cudaError_t e;
     switch (st) {
-      case 0: launch_stage<0>(p, nb, s); break;
-      case 1: launch_stage<1>(p, nb, s); break;
-      case 2: launch_stage<2>(p, nb, s); break;
-      case 3: launch_stage<3>(p, nb, s); break;
-      case 4: launch_stage<4>(p, nb, s); break;
-      case 5: launch_stage<5>(p, nb, s); break;
-      case 6: launch_stage<6>(p, nb, s); break;
-      default: launch_stage<7>(p, nb, s); break;
+      case 0: e = launch_stage<0>(p, ch, s); break;
+      case 1: e = launch_stage<1>(p, ch, s); break;
+      case 2: e = launch_stage<2>(p, ch, s); break;
+      case 3: e = launch_stage<3>(p, ch, s); break;
+      case 4: e = launch_stage<4>(p, ch, s); break;
+      case 5: e = launch_stage<5>(p, ch, s); break;
+      case 6: e = launch_stage<6>(p, ch, s); break;
+      default: e = launch_stage<7>(p, ch, s); break;
     }
-    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = launch(quant_reduce_kernel, (unsigned)p.count, 0, true, p, s);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -462,22 +457,19 @@ int64_t quant_blocks_for(int64_t N, int64_t K) {
   return (nquads + kQuadsPerBlock - 1) / kQuadsPerBlock;
 }
 
-// Workspace: [tickets: 16 B per tensor, padded to 256 B][partials of tensor 0][tensor 1]...
+// Workspace: the tile partials of tensor 0, then of tensor 1, ...
 size_t quant_workspace_bytes(const ifq_qtensor* t, int count) {
-  size_t bytes = ((size_t)count * 16 + 255) / 256 * 256;
+  size_t bytes = 0;
   for (int i = 0; i < count; ++i) bytes += (size_t)quant_blocks_for(t[i].N, t[i].K) * sizeof(QPartial);
   return bytes;
 }
 
 cudaError_t launch_quantize(const ifq_qtensor* t, int count, int T, void* ws, uint32_t* dev_status, cudaStream_t s) {
   QParams p;
-  size_t ticket_bytes = 0;
-  const int64_t blocks = fill_qparams(t, count, ws, p, &ticket_bytes);
+  const int64_t tiles = fill_qparams(t, count, ws, p);
   p.status = dev_status;
-  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaMemsetAsync(ws, 0, ticket_bytes, s);
-  if (e != cudaSuccess) return e;
-  return launch_stages(p, blocks, 0, T, s);
+  if (tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  return launch_stages(p, 0, T, false, s);
 }
 
 size_t widely_linear_quant_workspace_bytes(const ifq_wl_layer* Ls, int count) {
@@ -491,8 +483,7 @@ cudaError_t launch_widely_linear_quantize(const ifq_wl_layer* Ls, int count, int
   ifq_qtensor t[IFQ_MAX_GROUP];
   fused_tensors(Ls, count, t);
   QParams p;
-  size_t ticket_bytes = 0;
-  const int64_t blocks = fill_qparams(t, 2 * count, ws, p, &ticket_bytes);
+  const int64_t tiles = fill_qparams(t, 2 * count, ws, p);
   p.status = dev_status;
   FParams f;
   memset(&f, 0, sizeof(f));
@@ -509,13 +500,14 @@ cudaError_t launch_widely_linear_quantize(const ifq_wl_layer* Ls, int count, int
     a.w = p.t[2 * i + 1];
     fblocks += a.u.nblocks;
   }
-  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaMemsetAsync(ws, 0, ticket_bytes, s);
-  if (e != cudaSuccess) return e;
+  if (tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   widely_linear_quant1_kernel<<<(unsigned)fblocks, kQThreads, 0, s>>>(f);
-  e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_stages(p, blocks, 1, T, s);
+  p.stage = 0;
+  e = launch(quant_reduce_kernel, (unsigned)p.count, 0, true, p, s);
+  if (e != cudaSuccess) return e;
+  return launch_stages(p, 1, T, true, s);
 }
 
 // Scratch of ifq_quantize_pack_static, for callers that cannot hand over device

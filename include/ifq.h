@@ -146,8 +146,8 @@ ifq_status ifq_quantize_pack(const ifq_qtensor* tensors, int count, int T, void*
  * IFQ_QUANT_STATIC_SCRATCH_BYTES (2 MiB: 32 bytes per 4096 complex weights,
  * about 2.7e8 complex weights per call in total); larger calls return
  * IFQ_ERR_STATIC_LIMIT before anything is launched.
- * The part of the scratch that must start at zero (the per-tensor tickets) is
- * cleared by every call with an asynchronous memset on `stream`.
+ * The scratch needs no initial contents: every call writes each part of it
+ * before reading it.
  * The first call on a device (with that device current) looks up the array's
  * device address once (cudaGetSymbolAddress) and may load the library's device
  * code; make that first call before anything that must not see such set-up,
