@@ -306,6 +306,33 @@ def decode_b16(block, reps=20):
 
 
 # ---------------------------------------------------------------- dense comparator
+def decode_rope(block, reps=20):
+    """The block's decode product at B = 1 with the complex rotary code applied in the epilogue of the
+    q and k projections (layers 0 and 1; rot = e^{i pos omega_n}), after an L2 flush, through the C ABI.
+    Reported beside the plain decode time: the rotation adds 8 bytes read per rotated output."""
+    layers = [dict(d) for d in block.gemv_layers]
+    pos = 1234
+    for i in (0, 1):
+        N = layers[i]["N"]
+        omega = 10000.0 ** (-torch.arange(N, dtype=torch.float64) / N)
+        layers[i]["rot_re"] = torch.cos(pos * omega).to(torch.float32).reshape(1, N).to(block.dev)
+        layers[i]["rot_im"] = torch.sin(pos * omega).to(torch.float32).reshape(1, N).to(block.dev)
+    ls = Q.LayerSet(layers)
+    times = []
+    for k in range(reps + 3):
+        block.flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        Q.ifq_gemv(ls, block.T, 1, workspace=block.gemv_ws, dev_status=block.status)
+        b.record()
+        torch.cuda.synchronize()
+        if k >= 3:
+            times.append(a.elapsed_time(b) * 1e-3)
+    assert int(block.status.item()) == 0, "device status set by the rotated decode"
+    t = statistics.median(times)
+    return {"us": t * 1e6, "rotated_layers": ["q", "k"], "GBps": block.gemv_bytes(1) / t / 1e9}
+
+
 def fused_convert_quantize(block, reps=10):
     """Conversion fused with stage 1 of the quantizer (one call for the block's seven layers), timed
     with CUDA events; its inputs (3.2 GB of R) are far larger than L2.  Reported beside the two-pass
@@ -481,6 +508,9 @@ def run_ours(args):
         cpu = oracle_decode_sample(seconds_budget=args.cpu_seconds)
     b16 = decode_b16(block) if rank == 0 else None
     fused = fused_convert_quantize(block) if rank == 0 else None
+    rope = decode_rope(block) if rank == 0 else None
+    if rope is not None:
+        rope["plain_decode_us"] = t_gemv * 1e6
     if fused is not None:
         fused["two_pass_us"] = (t_conv + t_quant) * 1e6
         fused["speedup_over_two_pass"] = (t_conv + t_quant) / (fused["us"] * 1e-6)
@@ -540,6 +570,7 @@ def run_ours(args):
         "e2e": e2e,
         "decode_b16": b16,
         "fused_convert_quantize": fused,
+        "decode_rope": rope,
         "dense_bf16_comparator": dense,
         "gpu_launches": block.launches_per_step() * args.steps,
         "clocks": clk,

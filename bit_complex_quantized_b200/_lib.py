@@ -62,7 +62,7 @@ class Layer(ctypes.Structure):
     _fields_ = [("codes_u", ctypes.c_void_p), ("scales_u", ctypes.c_void_p), ("codes_w", ctypes.c_void_p),
                 ("scales_w", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
                 ("x_re", ctypes.c_void_p), ("x_im", ctypes.c_void_p), ("y_re", ctypes.c_void_p),
-                ("y_im", ctypes.c_void_p)]
+                ("y_im", ctypes.c_void_p), ("rot_re", ctypes.c_void_p), ("rot_im", ctypes.c_void_p)]
 
 
 _lib = None
@@ -186,7 +186,9 @@ def _layers(layers):
                        None if d.get("codes_w") is None else d["codes_w"].data_ptr(),
                        None if d.get("scales_w") is None else d["scales_w"].data_ptr(),
                        d["N"], d["K"], d["x_re"].data_ptr(), d["x_im"].data_ptr(), d["y_re"].data_ptr(),
-                       d["y_im"].data_ptr())
+                       d["y_im"].data_ptr(),
+                       None if d.get("rot_re") is None else d["rot_re"].data_ptr(),
+                       None if d.get("rot_im") is None else d["rot_im"].data_ptr())
     return arr
 
 
@@ -213,8 +215,9 @@ def ifq_gemv_workspace_bytes(layers, T, B):
 
 def ifq_gemv(layers, T, B, workspace=None, dev_status=None, stream=None, workspace_bytes=None):
     """layers: list of dicts with codes_u, scales_u, codes_w, scales_w (or None), N, K,
-    x_re, x_im (bf16 [B][K]), y_re, y_im (float32 [B][N]).  workspace: a device
-    buffer of ifq_gemv_workspace_bytes() bytes, zero-filled before its first use."""
+    x_re, x_im (bf16 [B][K]), y_re, y_im (float32 [B][N]), and optionally rot_re, rot_im
+    (float32 [B][N]: each output is multiplied by rot_re + i rot_im).  workspace: a device
+    buffer of ifq_gemv_workspace_bytes() bytes (no initial contents needed)."""
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     if workspace_bytes is not None:
         nbytes = workspace_bytes

@@ -32,11 +32,12 @@ ifq_status check_layers(const ifq_layer* L, int count, int T) {
     const ifq_layer& l = L[i];
     if (!l.codes_u || !l.scales_u || !l.x_re || !l.x_im || !l.y_re || !l.y_im) return IFQ_ERR_NULL;
     if ((l.codes_w == nullptr) != (l.scales_w == nullptr)) return IFQ_ERR_NULL;
+    if ((l.rot_re == nullptr) != (l.rot_im == nullptr)) return IFQ_ERR_NULL;
     if (l.N < 1 || l.K < 64 || (l.K % 64) != 0) return IFQ_ERR_SHAPE;
     if (l.N > (int64_t)1 << 30 || l.K > (int64_t)1 << 30) return IFQ_ERR_SHAPE;
     if (!aligned16(l.codes_u) || (l.codes_w && !aligned16(l.codes_w)) || !aligned16(l.x_re) || !aligned16(l.x_im) ||
         !aligned16(l.y_re) || !aligned16(l.y_im) || (reinterpret_cast<uintptr_t>(l.scales_u) & 3u) ||
-        (reinterpret_cast<uintptr_t>(l.scales_w) & 3u))
+        (reinterpret_cast<uintptr_t>(l.scales_w) & 3u) || (l.rot_re && (!aligned16(l.rot_re) || !aligned16(l.rot_im))))
       return IFQ_ERR_ALIGN;
   }
   return IFQ_OK;

@@ -67,6 +67,7 @@ struct __align__(64) GemmArgs {
   CUtensorMap tmap_codes[2];  // u8 [T*N][K/4]: box {16, 64}
   const float* scales[2];
   float* y[2];
+  const float* rot[2];  // optional epilogue rotation [M][N] (re, im), or null
   int64_t N, K, M;
   int T, nbranch;
   uint32_t* status;
@@ -280,21 +281,49 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     // all epilogue warps have finished the tile's y: store it (rows of 64 outputs, float4)
     asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
     if (!__shfl_sync(0xffffffffu, *abort, 0)) {
-      const int e = threadIdx.x - kExpWarps * 32;  // 0..127
+      const int e = threadIdx.x - kExpWarps * 32;  // 0..255
       const bool vec = (a.N & 3) == 0 && n0 + BN <= a.N;
-      for (int idx = e; idx < 2 * BM * (BN / 4); idx += kEpiWarps * 32) {
-        const int pl = idx / (BM * (BN / 4)), rem = idx - pl * (BM * (BN / 4));
-        const int tok = rem / (BN / 4), c4 = rem - tok * (BN / 4);
+      for (int idx = e; idx < BM * (BN / 4); idx += kEpiWarps * 32) {
+        const int tok = idx / (BN / 4), c4 = idx - tok * (BN / 4);
         const int64_t m = m0 + tok;
         if (m >= a.M) continue;
-        const float4 v4 = *reinterpret_cast<const float4*>(ys + pl * BM * BN + tok * BN + 4 * c4);
-        float* dst = a.y[pl] + m * a.N + n0 + 4 * c4;
+        const float4 r4 = *reinterpret_cast<const float4*>(ys + tok * BN + 4 * c4);
+        const float4 i4 = *reinterpret_cast<const float4*>(ys + BM * BN + tok * BN + 4 * c4);
+        float vr[4] = {r4.x, r4.y, r4.z, r4.w}, vi[4] = {i4.x, i4.y, i4.z, i4.w};
+        const int64_t o = m * a.N + n0 + 4 * c4;
+        const int nv = vec ? 4 : (int)(a.N - (n0 + 4 * c4) < 4 ? a.N - (n0 + 4 * c4) : 4);  // valid outputs
+        if (a.rot[0]) {  // complex RoPE: times rot[m][n]
+          float cr[4] = {1.f, 1.f, 1.f, 1.f}, ci[4] = {0.f, 0.f, 0.f, 0.f};
+          if (vec) {
+            const float4 c = __ldg(reinterpret_cast<const float4*>(a.rot[0] + o));
+            const float4 d = __ldg(reinterpret_cast<const float4*>(a.rot[1] + o));
+            cr[0] = c.x; cr[1] = c.y; cr[2] = c.z; cr[3] = c.w;
+            ci[0] = d.x; ci[1] = d.y; ci[2] = d.z; ci[3] = d.w;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              if (j < nv) {
+                cr[j] = __ldg(a.rot[0] + o + j);
+                ci[j] = __ldg(a.rot[1] + o + j);
+              }
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float r = cr[j] * vr[j] - ci[j] * vi[j], im = cr[j] * vi[j] + ci[j] * vr[j];
+            vr[j] = r;
+            vi[j] = im;
+          }
+        }
         if (vec) {
-          *reinterpret_cast<float4*>(dst) = v4;
+          *reinterpret_cast<float4*>(a.y[0] + o) = make_float4(vr[0], vr[1], vr[2], vr[3]);
+          *reinterpret_cast<float4*>(a.y[1] + o) = make_float4(vi[0], vi[1], vi[2], vi[3]);
         } else {
-          const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
           for (int j = 0; j < 4; ++j)
-            if (n0 + 4 * c4 + j < a.N) dst[j] = vv[j];
+            if (j < nv) {
+              a.y[0][o + j] = vr[j];
+              a.y[1][o + j] = vi[j];
+            }
         }
       }
     }
@@ -369,6 +398,8 @@ cudaError_t launch_gemm(const ifq_layer* Ls, int count, int T, int64_t M, uint32
     a.scales[1] = L.scales_w;
     a.y[0] = L.y_re;
     a.y[1] = L.y_im;
+    a.rot[0] = L.rot_re;
+    a.rot[1] = L.rot_im;
     bool ok = make_map_2d(&a.tmap_x[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L.x_re, (uint64_t)L.K, (uint64_t)M,
                           (uint64_t)L.K * 2, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
               make_map_2d(&a.tmap_x[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L.x_im, (uint64_t)L.K, (uint64_t)M,

@@ -45,6 +45,7 @@ struct GemvLayerArg {
   const float* scales[2];
   const uint16_t* x[2];  // re, im
   float* y[2];           // re, im
+  const float* rot[2];   // optional epilogue rotation [B][N] (re, im), or null
   int64_t N;
   int64_t K;
   int64_t block_begin;
@@ -77,6 +78,18 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
+}
+
+// Output element idx = tok * N + n, times the optional rotation rot[idx] (complex RoPE).
+__device__ __forceinline__ void store_y(const GemvLayerArg& L, int64_t idx, float yr, float yi) {
+  if (L.rot[0]) {
+    const float cr = __ldg(L.rot[0] + idx), ci = __ldg(L.rot[1] + idx);
+    const float r = cr * yr - ci * yi, i = cr * yi + ci * yr;
+    yr = r;
+    yi = i;
+  }
+  L.y[0][idx] = yr;
+  L.y[1][idx] = yi;
 }
 
 // NT: MMA n-tiles (8 columns = 4 tokens each); MI: code matrices per pass over a chunk.
@@ -206,14 +219,8 @@ __global__ void __launch_bounds__(32 * kWarps) gemv_kernel(const __grid_constant
   for (int nt = 0; nt < NT; ++nt) {
     const int tok = nt * 4 + tq;
     if (tok < p.B) {
-      if (okA) {
-        L.y[0][(int64_t)tok * L.N + rowA] = yr[nt][0];
-        L.y[1][(int64_t)tok * L.N + rowA] = yi[nt][0];
-      }
-      if (okB) {
-        L.y[0][(int64_t)tok * L.N + rowB] = yr[nt][1];
-        L.y[1][(int64_t)tok * L.N + rowB] = yi[nt][1];
-      }
+      if (okA) store_y(L, (int64_t)tok * L.N + rowA, yr[nt][0], yi[nt][0]);
+      if (okB) store_y(L, (int64_t)tok * L.N + rowB, yr[nt][1], yi[nt][1]);
     }
   }
 }
@@ -244,6 +251,8 @@ cudaError_t launch_gemv(const ifq_layer* Ls, int count, int T, int B, uint32_t* 
     a.x[1] = Ls[i].x_im;
     a.y[0] = Ls[i].y_re;
     a.y[1] = Ls[i].y_im;
+    a.rot[0] = Ls[i].rot_re;
+    a.rot[1] = Ls[i].rot_im;
     a.N = Ls[i].N;
     a.K = Ls[i].K;
     p.order[i] = i;

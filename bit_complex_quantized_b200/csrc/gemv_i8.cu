@@ -62,6 +62,7 @@ struct I8Layer {
   const float* scales[2];
   const uint16_t* x[2];
   float* y[2];
+  const float* rot[2];    // optional epilogue rotation [N] (re, im), or null
   uint4* frag;            // [blocks][8 chunks][32 lanes][4]: a lane's 8 k-step fragments of a chunk, contiguous
   double* bsum;           // [blocks][9][2]: exact sums of v over the block's first c chunks, per plane
   int* bexp;              // [blocks]
@@ -232,6 +233,18 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(const __grid_co
 }
 
 // ---------------------------------------------------------------- main kernel
+// Output n of the token, times the optional rotation rot[n] (complex RoPE).
+__device__ __forceinline__ void store_y(const I8Layer& L, int64_t n, float yr, float yi) {
+  if (L.rot[0]) {
+    const float cr = __ldg(L.rot[0] + n), ci = __ldg(L.rot[1] + n);
+    const float r = cr * yr - ci * yi, i = cr * yi + ci * yr;
+    yr = r;
+    yi = i;
+  }
+  L.y[0][n] = yr;
+  L.y[1][n] = yi;
+}
+
 // A piece: chunks [ch, ch + len) of one (tile, matrix) row block, inside one K block.
 struct Piece {
   int li;
@@ -594,10 +607,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_i8_kernel(const 
         if (tq == 0) {
 #pragma unroll
           for (int r = 0; r < 2; ++r)
-            if (row0 + g + 8 * r < L.N) {
-              L.y[0][row0 + g + 8 * r] = (float)yr[r];
-              L.y[1][row0 + g + 8 * r] = (float)yi[r];
-            }
+            if (row0 + g + 8 * r < L.N) store_y(L, row0 + g + 8 * r, (float)yr[r], (float)yi[r]);
         }
       } else {
         const int64_t slot0 = cur.tile * tc;
@@ -630,8 +640,7 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_i8_kernel(const 
               if (cn <= c) break;  // cannot happen: portions are non-empty and ordered
               c = cn;
             }
-            L.y[0][row0 + lane] = ar;
-            L.y[1][row0 + lane] = ai;
+            store_y(L, row0 + lane, ar, ai);
           }
           if (lane == 0) L.tickets[cur.tile] = 0u;
         }
@@ -713,6 +722,8 @@ cudaError_t launch_cap(const ifq_layer* Ls, int count, int T, void* ws, uint32_t
     a.x[1] = Ls[i].x_im;
     a.y[0] = Ls[i].y_re;
     a.y[1] = Ls[i].y_im;
+    a.rot[0] = Ls[i].rot_re;
+    a.rot[1] = Ls[i].rot_im;
     a.N = Ls[i].N;
     a.K = Ls[i].K;
     a.tiles = (int32_t)((a.N + 15) / 16);

@@ -223,7 +223,21 @@ ifq_status ifq_widely_linear_quantize_pack(const ifq_wl_layer* layers, int count
  *   N, K                outputs, inputs: N >= 1, K >= 64, K % 64 == 0
  *   x_re, x_im          [rows][K] bf16 bit patterns, device, 16-byte aligned
  *   y_re, y_im          [rows][N] float32, device, overwritten
+ *   rot_re, rot_im      optional epilogue rotation, both NULL = none: when set,
+ *                       output [r][n] is multiplied by the complex number
+ *                       rot_re[r][n] + i rot_im[r][n] ([rows][N] float32,
+ *                       device, 16-byte aligned) before it is stored.  This is
+ *                       the complex rotary position encoding of the q and k
+ *                       projections, one complex multiply per output ("iFairy
+ *                       article" §三; "iFairy talk notes" §2.1.3): the caller
+ *                       passes e^{i theta} for each token position and output.
+ *                       Setting only one of the two is IFQ_ERR_NULL.
  * rows = B for ifq_gemv and M for ifq_gemm.
+ *
+ * The attention score of the complex model, Re(q^T conj(k)) ("Fairy2i write-up"
+ * §2.2; "iFairy talk notes" §2.1.4), equals the real dot product of the stacked
+ * vectors [q_re, q_im] and [k_re, k_im], so the planar outputs feed a standard
+ * real attention kernel directly; the library has no score kernel of its own.
  * ------------------------------------------------------------------------- */
 typedef struct {
   const uint8_t* codes_u;
@@ -236,6 +250,8 @@ typedef struct {
   const uint16_t* x_im;
   float* y_re;
   float* y_im;
+  const float* rot_re;
+  const float* rot_im;
 } ifq_layer;
 
 /* Decode product for B = 1..IFQ_MAX_GEMV_BATCH tokens per layer; all `count`

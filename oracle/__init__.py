@@ -8,7 +8,9 @@ Sources, by page and section:
   * "Fairy2i write-up" (hotelren.com): §2.1 widely-linear transform,
     §3.1 phase rule, §3.2 axis scales, §4.1 recursive residual, §4.2 product.
   * "iFairy article" (bestcxt.com): §二.1 codebook, §二.2 multiplication-free GEMM.
-  * "iFairy talk notes" (43b.com.cn): §2.2.2 phase rule, §2.3.1 x i = swap + negate.
+  * "iFairy talk notes" (43b.com.cn): §2.2.2 phase rule, §2.3.1 x i = swap + negate,
+    §2.1.3 rotary position code, §2.1.4 real-part attention score.
+  * "iFairy article" §三: complex rotary position code as one complex multiply.
 """
 from .phasequant import (  # noqa: F401
     CODEBOOK,
@@ -26,6 +28,8 @@ from .phasequant import (  # noqa: F401
     product,
     product_rows,
     tolerance_bound,
+    rotate_outputs,
+    score,
     near_boundary_mask,
     bf16_round,
     bf16_bits_to_f64,

@@ -271,6 +271,26 @@ def tolerance_bound(scales_u, scales_w, x_re, x_im, rel=1e-5):
 
 
 # ---------------------------------------------------------------------------
+# Adjacent decode-block steps: complex rotary position encoding of the q / k
+# projections ("iFairy article" §三: in the complex domain the rotation is one
+# complex multiplication; "iFairy talk notes" §2.1.3) and the attention score
+# Re(q^T conj(k)) ("Fairy2i write-up" §2.2, item 2; "iFairy talk notes" §2.1.4).
+# The pages fix no frequencies: the rotation factors are inputs.
+# ---------------------------------------------------------------------------
+def rotate_outputs(y, rot_re, rot_im):
+    """y (complex [rows][N]) times the per-output rotation rot_re + i rot_im, in complex128."""
+    rot = np.asarray(rot_re, np.float64) + 1j * np.asarray(rot_im, np.float64)
+    return np.asarray(y, np.complex128) * rot
+
+
+def score(q, k):
+    """Real part of the Hermitian inner product: Re(sum_j q_j conj(k_j)), over the last axis."""
+    q = np.asarray(q, np.complex128)
+    k = np.asarray(k, np.complex128)
+    return np.real(np.sum(q * np.conj(k), axis=-1))
+
+
+# ---------------------------------------------------------------------------
 # bf16 helpers (exact conversions only)
 # ---------------------------------------------------------------------------
 def bf16_bits_to_f64(bits):

@@ -168,3 +168,17 @@ def test_fused_convert_quantize_argument_errors():
     assert call(arr, ws=None) == 6 and call(arr, nb=need - 1) == 6
     assert call(arr, ws=FAKE + 8) == 3
     assert lib.ifq_widely_linear_quantize_workspace_bytes((L.WlLayer * 1)(_wl(cols=12)), 1, 2) == 0
+
+
+def test_rotation_argument_errors():
+    lib = Q.load()
+    one = lambda **kw: (L.Layer * 1)(_layer(**kw))  # noqa: E731
+    base = _layer()
+    rot = (L.Layer * 1)(L.Layer(base.codes_u, base.scales_u, None, None, 64, 128, FAKE, FAKE, FAKE, FAKE,
+                                FAKE, None))
+    assert lib.ifq_gemv(rot, 1, 1, 1, FAKE, 1 << 30, None, None) == 1     # one of the two planes missing
+    assert lib.ifq_gemm(rot, 1, 1, 128, None, None) == 1
+    mis = (L.Layer * 1)(L.Layer(base.codes_u, base.scales_u, None, None, 64, 128, FAKE, FAKE, FAKE, FAKE,
+                                FAKE + 4, FAKE))
+    assert lib.ifq_gemv(mis, 1, 1, 1, FAKE, 1 << 30, None, None) == 3
+    assert one() is not None

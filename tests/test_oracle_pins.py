@@ -456,3 +456,58 @@ def test_c_near_boundary_flags_match_numpy():
     a, b = O.residual_after(wr, wi, [O.unpack_codes(codes[0])], [tuple(scales[0])])
     want = O.near_boundary_mask(a, b, float(np.sum(scales[0].astype(np.float64))))
     np.testing.assert_array_equal(near.reshape(16, 64).astype(bool), want)
+
+
+# ---------------------------------------------------------------- rotation and score
+def test_rotation_by_i_is_swap_and_negate():
+    """x i = (-Im x) + i Re x exactly ("iFairy talk notes" §2.3.1), element by element."""
+    rng = np.random.default_rng(21)
+    y = rng.standard_normal((3, 17)) + 1j * rng.standard_normal((3, 17))
+    got = O.rotate_outputs(y, np.zeros((3, 17)), np.ones((3, 17)))
+    np.testing.assert_array_equal(got.real, -y.imag)
+    np.testing.assert_array_equal(got.imag, y.real)
+    np.testing.assert_array_equal(O.rotate_outputs(y, np.ones((3, 17)), np.zeros((3, 17))), y)
+
+
+def test_rotation_keeps_modulus_and_inverts():
+    rng = np.random.default_rng(22)
+    y = rng.standard_normal((4, 33)) + 1j * rng.standard_normal((4, 33))
+    th = rng.uniform(-np.pi, np.pi, (4, 33))
+    z = O.rotate_outputs(y, np.cos(th), np.sin(th))
+    np.testing.assert_allclose(np.abs(z), np.abs(y), rtol=1e-14)
+    back = O.rotate_outputs(z, np.cos(-th), np.sin(-th))
+    np.testing.assert_allclose(back, y, rtol=1e-13, atol=1e-13)
+    # the phase advances by theta: arg(z) - arg(y) = theta (mod 2 pi)
+    d = np.angle(z) - np.angle(y) - th
+    np.testing.assert_allclose(np.angle(np.exp(1j * d)), 0.0, atol=1e-12)
+
+
+def test_score_is_polar_form_and_real_special_case():
+    """Re(q^T conj(k)) = sum |q||k| cos(arg q - arg k); for real vectors the ordinary dot product;
+    symmetric in q and k."""
+    rng = np.random.default_rng(23)
+    q = rng.standard_normal(64) + 1j * rng.standard_normal(64)
+    k = rng.standard_normal(64) + 1j * rng.standard_normal(64)
+    polar = float(np.sum(np.abs(q) * np.abs(k) * np.cos(np.angle(q) - np.angle(k))))
+    assert abs(O.score(q, k) - polar) <= 1e-12 * float(np.sum(np.abs(q) * np.abs(k)))
+    assert O.score(q, k) == pytest.approx(O.score(k, q), rel=1e-15, abs=1e-15)
+    a, b = rng.standard_normal(50), rng.standard_normal(50)
+    assert O.score(a + 0j, b + 0j) == pytest.approx(float(sum(float(u) * float(v) for u, v in zip(a, b))),
+                                                   rel=1e-12)
+
+
+def test_score_of_rotated_pair_depends_on_position_difference_only():
+    """Rotating q by theta_q and k by theta_k per dimension, with theta = position * omega, leaves a
+    score that depends on the positions only through their difference (the point of the rotary code)."""
+    rng = np.random.default_rng(24)
+    d = 32
+    omega = 10000.0 ** (-np.arange(d) / d)
+    q = rng.standard_normal(d) + 1j * rng.standard_normal(d)
+    k = rng.standard_normal(d) + 1j * rng.standard_normal(d)
+
+    def rot(v, pos):
+        return O.rotate_outputs(v, np.cos(pos * omega), np.sin(pos * omega))
+    s1 = O.score(rot(q, 7), rot(k, 3))
+    s2 = O.score(rot(q, 104), rot(k, 100))
+    assert s1 == pytest.approx(s2, rel=1e-10, abs=1e-10)
+    assert O.score(rot(q, 5), rot(k, 5)) == pytest.approx(O.score(q, k), rel=1e-12, abs=1e-12)
