@@ -306,6 +306,32 @@ def decode_b16(block, reps=20):
 
 
 # ---------------------------------------------------------------- dense comparator
+def dequantize_block(block, reps=10):
+    """bf16 dequantized weights of the block's 14 tensors (the forward weights of quantization-aware
+    training), one ifq_dequantize call, CUDA events; reads T/4 B of codes and writes 4 B of bf16 per
+    complex entry (910 MB of writes: larger than L2)."""
+    ts = []
+    for (cu, su), spec in zip(block.codes, [l for l in block.cfg.layers for _ in range(2)]):
+        ts.append((cu, su, torch.empty((spec.N, spec.K), dtype=torch.int16, device=block.dev),
+                   torch.empty((spec.N, spec.K), dtype=torch.int16, device=block.dev)))
+    times = []
+    for k in range(reps + 3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        Q.ifq_dequantize(ts, block.T)
+        b.record()
+        torch.cuda.synchronize()
+        if k >= 3:
+            times.append(a.elapsed_time(b) * 1e-3)
+    t = statistics.median(times)
+    entries = 2 * sum(l.N * l.K for l in block.cfg.layers)
+    nbytes = entries * (block.T / 4 + 4)
+    gbs = nbytes / t / 1e9
+    del ts
+    return {"us": t * 1e6, "algorithmic_bytes": int(nbytes), "GBps": gbs,
+            "frac_of_hbm": gbs / float(peaks()[0]["hbm_gbs"])}
+
+
 def decode_rope(block, reps=20):
     """The block's decode product at B = 1 with the complex rotary code applied in the epilogue of the
     q and k projections (layers 0 and 1; rot = e^{i pos omega_n}), after an L2 flush, through the C ABI.
@@ -509,6 +535,7 @@ def run_ours(args):
     b16 = decode_b16(block) if rank == 0 else None
     fused = fused_convert_quantize(block) if rank == 0 else None
     rope = decode_rope(block) if rank == 0 else None
+    dq = dequantize_block(block) if rank == 0 else None
     if rope is not None:
         rope["plain_decode_us"] = t_gemv * 1e6
     if fused is not None:
@@ -571,6 +598,7 @@ def run_ours(args):
         "decode_b16": b16,
         "fused_convert_quantize": fused,
         "decode_rope": rope,
+        "dequantize_bf16": dq,
         "dense_bf16_comparator": dense,
         "gpu_launches": block.launches_per_step() * args.steps,
         "clocks": clk,
@@ -677,6 +705,17 @@ def run_case(args):
         def fn():
             Q.ifq_widely_linear_quantize_pack(wl, 2, wsb)
         label = "fused convert + quantize c3 gate T=2"
+    elif args.case == "dequant":
+        cfg = W.config("c3")
+        spec = cfg.layers[4]
+        cb = torch.randint(0, 256, (2, spec.N, spec.K // 4), dtype=torch.uint8, device=dev, generator=g)
+        sc = torch.full((2, 2), 0.01, device=dev)
+        outp = [torch.empty((spec.N, spec.K), dtype=torch.int16, device=dev) for _ in range(2)]
+        nbytes = spec.N * spec.K * (2 / 4 + 4)
+
+        def fn():
+            Q.ifq_dequantize([(cb, sc, outp[0], outp[1])], 2)
+        label = "dequantize bf16 c3 gate T=2"
     elif args.case == "convert":
         cfg = W.config("c3")
         spec = cfg.layers[4]
@@ -714,7 +753,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--case", choices=["gemv", "gemm", "quant", "convert", "wlq"], default=None)
+    ap.add_argument("--case", choices=["gemv", "gemm", "quant", "convert", "wlq", "dequant"], default=None)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--workload", choices=["c3", "c5"], default="c5", help="layer set of --case gemv")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

@@ -15,6 +15,7 @@ from ._lib import (  # noqa: F401
     IfqError,
     LayerSet,
     LIB_PATH,
+    ifq_dequantize,
     ifq_gemm,
     ifq_gemv,
     ifq_gemv_workspace_bytes,

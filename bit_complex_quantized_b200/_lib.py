@@ -28,6 +28,7 @@ EXPORTED = (
     "ifq_quantize_pack_static",
     "ifq_widely_linear_quantize_workspace_bytes",
     "ifq_widely_linear_quantize_pack",
+    "ifq_dequantize",
     "ifq_gemv_workspace_bytes",
     "ifq_gemv",
     "ifq_gemm",
@@ -49,6 +50,11 @@ class IfqError(RuntimeError):
 class QTensor(ctypes.Structure):
     _fields_ = [("w_re", ctypes.c_void_p), ("w_im", ctypes.c_void_p), ("N", ctypes.c_int64),
                 ("K", ctypes.c_int64), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+class DqTensor(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int64), ("w_re", ctypes.c_void_p), ("w_im", ctypes.c_void_p)]
 
 
 class WlLayer(ctypes.Structure):
@@ -91,6 +97,8 @@ def load():
     lib.ifq_widely_linear_quantize_workspace_bytes.argtypes = [ctypes.POINTER(WlLayer), i32, i32]
     lib.ifq_widely_linear_quantize_pack.restype = i32
     lib.ifq_widely_linear_quantize_pack.argtypes = [ctypes.POINTER(WlLayer), i32, i32, vp, sz, vp, vp]
+    lib.ifq_dequantize.restype = i32
+    lib.ifq_dequantize.argtypes = [ctypes.POINTER(DqTensor), i32, i32, vp]
     lib.ifq_gemv_workspace_bytes.restype = sz
     lib.ifq_gemv_workspace_bytes.argtypes = [ctypes.POINTER(Layer), i32, i32, i32]
     lib.ifq_gemv.restype = i32
@@ -153,6 +161,16 @@ def ifq_quantize_pack_static(tensors, T, dev_status=None, stream=None):
     """As ifq_quantize_pack, with the library's fixed device scratch instead of a workspace."""
     arr = _qtensors(tensors)
     _check(load().ifq_quantize_pack_static(arr, len(tensors), T, _ptr(dev_status), _stream(stream)))
+
+
+def ifq_dequantize(tensors, T, stream=None):
+    """tensors: list of (codes u8 [T][N][K/4], scales f32 [T][2], w_re, w_im) with w_* bf16 [N][K]
+    (written): the dequantized weights sum_t (s_re,t Re b_t + i s_im,t Im b_t)."""
+    arr = (DqTensor * len(tensors))()
+    for i, (codes, scales, w_re, w_im) in enumerate(tensors):
+        arr[i] = DqTensor(codes.data_ptr(), scales.data_ptr(), w_re.shape[0], w_re.shape[1], w_re.data_ptr(),
+                          w_im.data_ptr())
+    _check(load().ifq_dequantize(arr, len(tensors), T, _stream(stream)))
 
 
 def _wl_layers(layers):

@@ -161,6 +161,24 @@ ifq_status ifq_widely_linear_quantize_pack(const ifq_wl_layer* layers, int count
   return from_cuda(ifq::launch_widely_linear_quantize(layers, count, T, workspace, dev_status, as_stream(stream)));
 }
 
+ifq_status ifq_dequantize(const ifq_dqtensor* tensors, int count, int T, ifq_stream_t stream) {
+  if (!tensors) return IFQ_ERR_NULL;
+  if (count < 1 || count > IFQ_MAX_GROUP) return IFQ_ERR_COUNT;
+  if (T < 1 || T > IFQ_MAX_STAGES) return IFQ_ERR_STAGES;
+  for (int i = 0; i < count; ++i) {
+    const ifq_dqtensor& t = tensors[i];
+    if (!t.codes || !t.scales || !t.w_re || !t.w_im) return IFQ_ERR_NULL;
+    if (t.N < 1 || t.K < 4 || (t.K % 4) != 0) return IFQ_ERR_SHAPE;
+    if (t.K > (int64_t)1 << 30 || t.N > ((int64_t)1 << 40) / t.K) return IFQ_ERR_SHAPE;
+    if (!aligned16(t.codes) || !aligned16(t.w_re) || !aligned16(t.w_im) ||
+        (reinterpret_cast<uintptr_t>(t.scales) & 3u))
+      return IFQ_ERR_ALIGN;
+  }
+  ifq_status st = check_device();
+  if (st != IFQ_OK) return st;
+  return from_cuda(ifq::launch_dequantize(tensors, count, T, as_stream(stream)));
+}
+
 size_t ifq_gemv_workspace_bytes(const ifq_layer* layers, int count, int T, int B) {
   if (check_layers(layers, count, T) != IFQ_OK || B < 1 || B > IFQ_MAX_GEMV_BATCH) return 0;
   return B == 1 ? ifq::gemv_i8_workspace_bytes(layers, count, T) : 0;

@@ -25,6 +25,9 @@ size_t widely_linear_quant_workspace_bytes(const ifq_wl_layer* L, int count);
 cudaError_t launch_widely_linear_quantize(const ifq_wl_layer* L, int count, int T, void* ws, uint32_t* dev_status,
                                           cudaStream_t s);
 
+// Dequantized bf16 weights for training (dequantize.cu).
+cudaError_t launch_dequantize(const ifq_dqtensor* t, int count, int T, cudaStream_t s);
+
 cudaError_t launch_gemv(const ifq_layer* L, int count, int T, int B, uint32_t* dev_status, cudaStream_t s);
 
 // B = 1 integer tensor-core path (gemv_i8.cu) and its workspace size.

@@ -210,6 +210,34 @@ ifq_status ifq_widely_linear_quantize_pack(const ifq_wl_layer* layers, int count
                                            size_t workspace_bytes, uint32_t* dev_status, ifq_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * ifq_dequantize  ("Fairy2i write-up" §3.2, §4.1; "iFairy talk notes" §2.2.1)
+ *
+ * The dequantized weight W_hat = sum_t (s_re,t Re b_t + i s_im,t Im b_t) of each
+ * tensor as bf16 planes, for the forward pass of quantization-aware training
+ * (the straight-through backward passes the gradient unchanged and needs no
+ * call).  Per entry the stage terms are added in float32 in stage order from +0
+ * and the sum is rounded once to bf16, nearest-even.
+ *
+ *   tensors[i].codes        [T][N][K/4] uint8, device, read-only
+ *   tensors[i].scales       [T][2] float32, device, read-only (4-byte aligned)
+ *   tensors[i].N, K         N >= 1, K >= 4, K % 4 == 0
+ *   tensors[i].w_re, w_im   [N][K] bf16 bit patterns, device, written
+ *   count                   1..IFQ_MAX_GROUP tensors, one launch
+ *   T                       1..IFQ_MAX_STAGES (the stages summed)
+ * Pointers must be 16-byte aligned (scales: 4-byte).
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  const uint8_t* codes;
+  const float* scales;
+  int64_t N;
+  int64_t K;
+  uint16_t* w_re;
+  uint16_t* w_im;
+} ifq_dqtensor;
+
+ifq_status ifq_dequantize(const ifq_dqtensor* tensors, int count, int T, ifq_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Product layers ("Fairy2i write-up" §2.1, §4.2; "iFairy article" §二.2)
  *
  *   y = sum_t ( U_hat_t x + W_hat_t conj(x) ),  per token,

@@ -25,6 +25,7 @@ from .phasequant import (  # noqa: F401
     pack_codes,
     unpack_codes,
     dequantize,
+    dequantize_bf16,
     product,
     product_rows,
     tolerance_bound,

@@ -235,6 +235,24 @@ def dequantize(packed, scales, rows=None):
     return acc
 
 
+def dequantize_bf16(packed, scales):
+    """Dequantized weights for training ("iFairy talk notes" §2.2.1), as the library states them:
+    per entry the stage terms +-s_re (real axis) or +-s_im (imaginary axis) are added in float32 in
+    stage order starting from +0, and each sum is rounded once to bf16 (nearest-even).  Returns
+    (re, im) float32 arrays holding bf16 values."""
+    packed = np.asarray(packed)
+    scales = np.asarray(scales, dtype=np.float32)
+    T = packed.shape[0]
+    K = packed.shape[-1] * 4
+    re = np.zeros(packed.shape[1:-1] + (K,), dtype=np.float32)
+    im = np.zeros_like(re)
+    for t in range(T):
+        br, bi = code_to_br_bi(unpack_codes(packed[t]))   # exactly one of the two is +-1
+        re = np.where(br != 0, re + np.where(br > 0, scales[t, 0], -scales[t, 0]).astype(np.float32), re)
+        im = np.where(bi != 0, im + np.where(bi > 0, scales[t, 1], -scales[t, 1]).astype(np.float32), im)
+    return bf16_round(re), bf16_round(im)
+
+
 def product_rows(codes_u, scales_u, codes_w, scales_w, x_re, x_im, rows=None):
     """y[b, n] = sum_t (U_hat_t x_b + W_hat_t conj(x_b)) for the selected rows (complex128).
 

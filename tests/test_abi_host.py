@@ -182,3 +182,14 @@ def test_rotation_argument_errors():
                                 FAKE + 4, FAKE))
     assert lib.ifq_gemv(mis, 1, 1, 1, FAKE, 1 << 30, None, None) == 3
     assert one() is not None
+
+
+def test_dequantize_argument_errors():
+    lib = Q.load()
+    ok = (L.DqTensor * 1)(L.DqTensor(FAKE, FAKE, 8, 64, FAKE, FAKE))
+    assert lib.ifq_dequantize(None, 1, 1, None) == 1
+    assert lib.ifq_dequantize(ok, 0, 1, None) == 9
+    assert lib.ifq_dequantize(ok, 1, 9, None) == 4
+    assert lib.ifq_dequantize((L.DqTensor * 1)(L.DqTensor(FAKE, FAKE, 8, 66, FAKE, FAKE)), 1, 1, None) == 2
+    assert lib.ifq_dequantize((L.DqTensor * 1)(L.DqTensor(FAKE, None, 8, 64, FAKE, FAKE)), 1, 1, None) == 1
+    assert lib.ifq_dequantize((L.DqTensor * 1)(L.DqTensor(FAKE, FAKE, 8, 64, FAKE + 2, FAKE)), 1, 1, None) == 3

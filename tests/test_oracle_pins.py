@@ -511,3 +511,33 @@ def test_score_of_rotated_pair_depends_on_position_difference_only():
     s2 = O.score(rot(q, 104), rot(k, 100))
     assert s1 == pytest.approx(s2, rel=1e-10, abs=1e-10)
     assert O.score(rot(q, 5), rot(k, 5)) == pytest.approx(O.score(q, k), rel=1e-12, abs=1e-12)
+
+
+# ---------------------------------------------------------------- dequantized training weights
+def test_dequantize_bf16_single_stage_is_the_rounded_codeword():
+    """T = 1: each entry is s_re * (+-1) or i s_im * (+-1) rounded to bf16, with the other part zero
+    (one of real and imaginary part is always zero: "iFairy article" §二.1)."""
+    rng = np.random.default_rng(41)
+    k = rng.integers(0, 4, (1, 5, 64))
+    packed = O.pack_codes(k)
+    sc = np.array([[0.0123456, 0.0345678]], np.float32)
+    re, im = O.dequantize_bf16(packed, sc)
+    exact = O.dequantize(packed, sc)
+    np.testing.assert_array_equal(re, O.bf16_round(exact.real.astype(np.float32)))
+    np.testing.assert_array_equal(im, O.bf16_round(exact.imag.astype(np.float32)))
+    assert np.all((re == 0) | (im == 0))
+    vals = {float(v) for v in np.abs(re[re != 0])} | {float(v) for v in np.abs(im[im != 0])}
+    assert vals == {float(O.bf16_round(np.float32(0.0123456))), float(O.bf16_round(np.float32(0.0345678)))}
+
+
+def test_dequantize_bf16_is_within_rounding_of_the_exact_sum():
+    rng = np.random.default_rng(42)
+    for T in (2, 3, 8):
+        k = rng.integers(0, 4, (T, 7, 32))
+        packed = O.pack_codes(k)
+        sc = (rng.uniform(0.001, 0.05, (T, 2))).astype(np.float32)
+        re, im = O.dequantize_bf16(packed, sc)
+        exact = O.dequantize(packed, sc)
+        tot = float(np.sum(sc, dtype=np.float64))
+        for got, want in ((re, exact.real), (im, exact.imag)):
+            assert np.all(np.abs(got - want) <= 2.0 ** -8 * np.abs(want) + 2.0 ** -20 * tot)
