@@ -56,8 +56,9 @@ static_assert(kPieceChunks * 256 == kKBlock, "a piece is at most one K block, an
 // [chunk][row][64 B] (lanes of a quarter warp read two adjacent 64-byte rows:
 // conflict-free).  Pieces of a row's last, partial block arrive by one bulk copy
 // per row as [row][512 B].
+// The scalars first and the tensor maps (read by the copy engine only) last, so the
+// fields a warp reads sit in few constant-cache lines.
 struct I8Layer {
-  CUtensorMap tmap[2];    // per branch: (64 B, row of [T][N], chunk in block, full block), box 64 x 16 x 8 x 1
   const uint8_t* codes[2];
   const float* scales[2];
   const uint16_t* x[2];
@@ -77,19 +78,21 @@ struct I8Layer {
   int32_t nbranch;
   int32_t nch;            // 256-wide K chunks per row
   int32_t nbf;            // full 2048-wide K blocks (streamed by tensor copies)
+  CUtensorMap tmap[2];    // per branch: (64 B, row of [T][N], chunk in block, full block), box 64 x 16 x 8 x 1
 };
 
 // Capacity kCap >= count: calls of up to 8 layers pass a small parameter block.
+// The call-wide scalars and the layer-begin tables lead, in the first constant-cache lines.
 template <int kCap>
 struct I8Params {
-  int64_t chunk_begin[kCap];  // copies of the layers' first chunk and first prep CTA, packed so that
-  int64_t prep_begin[kCap];   // the search for a layer touches one or two constant-cache lines
-  I8Layer L[kCap];
   int64_t total_chunks;
   int count;
   int T;
   int sms;  // > 0: CTA b works as CTA (b % sms) * (gridDim / sms) + b / sms
   uint32_t* status;
+  int64_t chunk_begin[kCap];  // copies of the layers' first chunk and first prep CTA, packed so that
+  int64_t prep_begin[kCap];   // the search for a layer touches one or two constant-cache lines
+  I8Layer L[kCap];
 };
 
 __device__ __forceinline__ void imma_16832(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
