@@ -286,23 +286,31 @@ def oracle_decode_sample(seconds_budget=12.0, rows_per_layer=256):
 
 
 # ---------------------------------------------------------------- decode at B = 16
-def decode_b16(block, reps=20):
-    """The block's decode product at B = 16 (the bf16 mma.sync path), after an L2 flush, through
-    the same grouped call; reported beside the step, not part of it."""
-    layers = block._layers(block.cfg, 16)
+def decode_batch(block, B, reps=20):
+    """The block's decode product at batch B (B <= 4: the integer path; B >= 5: bf16 mma.sync), after
+    an L2 flush, through the same grouped call; reported beside the step, not part of it."""
+    layers = Q.LayerSet(block._layers(block.cfg, B))
+    nws = Q.ifq_gemv_workspace_bytes(layers, block.T, B)
+    ws = torch.zeros(max(16, nws), dtype=torch.uint8, device=block.dev)
     times = []
     for i in range(reps + 3):
         block.flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        Q.ifq_gemv(layers, block.T, 16, dev_status=block.status)
+        Q.ifq_gemv(layers, block.T, B, workspace=ws, dev_status=block.status)
         b.record()
         torch.cuda.synchronize()
         if i >= 3:
             times.append(a.elapsed_time(b) * 1e-3)
     t = statistics.median(times)
-    nbytes = block.gemv_bytes(16)
-    return {"us": t * 1e6, "algorithmic_bytes": nbytes, "GBps": nbytes / t / 1e9}
+    nbytes = block.gemv_bytes(B)
+    gbs = nbytes / t / 1e9
+    return {"B": B, "us": t * 1e6, "algorithmic_bytes": nbytes, "GBps": gbs,
+            "frac_of_hbm": gbs / float(peaks()[0]["hbm_gbs"]), "path": "integer" if B <= 4 else "bf16"}
+
+
+def decode_b16(block, reps=20):
+    return decode_batch(block, 16, reps)
 
 
 # ---------------------------------------------------------------- dense comparator
@@ -533,6 +541,7 @@ def run_ours(args):
     if rank == 0 and ws == 1 and not args.skip_cpu_baseline:
         cpu = oracle_decode_sample(seconds_budget=args.cpu_seconds)
     b16 = decode_b16(block) if rank == 0 else None
+    batched = [decode_batch(block, B) for B in (2, 4, 8)] if rank == 0 else None
     fused = fused_convert_quantize(block) if rank == 0 else None
     rope = decode_rope(block) if rank == 0 else None
     dq = dequantize_block(block) if rank == 0 else None
@@ -596,6 +605,7 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "decode_b16": b16,
+        "decode_batched": batched,
         "fused_convert_quantize": fused,
         "decode_rope": rope,
         "dequantize_bf16": dq,

@@ -49,7 +49,8 @@ constexpr int kPieceChunks = 8;                // at most 8 chunks (256 K positi
 constexpr int kSlotBytes = 8192;               // one slot: 16 rows x 8 chunks x 64 bytes
 constexpr int kMainSmem = kWarps * 2 * kSlotBytes + kWarps * 2 * 8;
 constexpr int kPrepThreads = 128;                // one item (plane, position, 16-group) per thread of a chunk
-constexpr int kCtasPerSm = 3;
+// Resident CTAs per SM: three, or two for four tokens (their sums and fragments need more registers).
+constexpr int ctas_per_sm(int nb) { return nb >= 4 ? 2 : 3; }
 static_assert(kPieceChunks * 256 == kKBlock, "a piece is at most one K block, and one run of the int32 sums");
 
 // Slot layouts.  Pieces inside a full K block arrive by one 4-D tensor copy as
@@ -64,10 +65,10 @@ struct I8Layer {
   const uint16_t* x[2];
   float* y[2];
   const float* rot[2];    // optional epilogue rotation [N] (re, im), or null
-  uint4* frag;            // [blocks][8 chunks][32 lanes][4]: a lane's 8 k-step fragments of a chunk, contiguous
-  double* bsum;           // [blocks][9][2]: exact sums of v over the block's first c chunks, per plane
-  int* bexp;              // [blocks]
-  float* partials;        // [tiles][chunks per tile][16][2] (one slot per warp touching the tile)
+  uint4* frag;            // [blocks][8 chunks][NB][32 lanes][4]: a lane's 8 k-step fragments of a chunk, contiguous
+  double* bsum;           // [blocks][NB][9][2]: exact sums of v over the block's first c chunks, per plane
+  int* bexp;              // [blocks][NB]
+  float* partials;        // [tiles][chunks per tile][NB][16][2] (one slot per warp touching the tile)
   int* next;              // [tiles][chunks per tile]: end of the portion that starts at this chunk
   unsigned int* tickets;  // [tiles]: finished chunks of the tile
   int64_t N, K;
@@ -88,6 +89,7 @@ struct I8Params {
   int64_t total_chunks;
   int count;
   int T;
+  int B;    // tokens; the kernels are built for NB >= B and treat tokens B..NB-1 as zero
   int sms;  // > 0: CTA b works as CTA (b % sms) * (gridDim / sms) + b / sms
   uint32_t* status;
   int64_t chunk_begin[kCap];  // copies of the layers' first chunk and first prep CTA, packed so that
@@ -121,7 +123,7 @@ __device__ __forceinline__ int find_layer_by(const P& p, int64_t idx, bool prep)
 // block's exponent, then writes the digit fragments of its own chunk and the
 // exact sum of v up to its chunk's end (prefix sums at chunk boundaries).  The
 // first CTA of a layer also zeroes the layer's tile tickets.
-template <class P>
+template <class P, int NB>
 __global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(const __grid_constant__ P p) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ __align__(16) uint16_t xs[2][kKBlock];
@@ -140,6 +142,9 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(const __grid_co
   const int klen = (int)(L.K - k0 < kKBlock ? L.K - k0 : kKBlock);  // multiple of 64
   if (c * 256 >= klen) return;  // the block's last chunk lies before this one
 
+  for (int tok = 0; tok < NB; ++tok) {
+  if (tok > 0) __syncthreads();  // the previous token's use of xs, smax and ssum is over
+  const bool live = tok < p.B;   // tokens past the batch are zero
   unsigned int mx = 0;
 #pragma unroll
   for (int r = 0; r < kKBlock / (8 * kPrepThreads); ++r) {
@@ -147,7 +152,7 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(const __grid_co
     for (int pl = 0; pl < 2; ++pl) {
       const int idx = (r * kPrepThreads + tid) * 8;
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (idx < klen) v = __ldg(reinterpret_cast<const uint4*>(L.x[pl] + k0 + idx));
+      if (idx < klen && live) v = __ldg(reinterpret_cast<const uint4*>(L.x[pl] + (int64_t)tok * L.K + k0 + idx));
       *reinterpret_cast<uint4*>(&xs[pl][idx]) = v;
       const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -215,7 +220,8 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(const __grid_co
     const int tqs = (grp >> 2) & 3, w = grp & 3;
     const int ks = (w >> 1) * 4 + q;  // k-step within the chunk: (word pair, position)
     // a lane's fragments for chunk c: 8 k-steps x (b0, b1) = 64 contiguous bytes
-    uint32_t* fr = reinterpret_cast<uint32_t*>(L.frag + ((int64_t)b * 8 + c) * 32 * 4) + ks * 2 + (w & 1);
+    uint32_t* fr =
+        reinterpret_cast<uint32_t*>(L.frag + (((int64_t)b * 8 + c) * NB + tok) * 32 * 4) + ks * 2 + (w & 1);
 #pragma unroll
     for (int d = 0; d < 4; ++d) fr[((pl * 4 + d) * 4 + tqs) * 16] = dig[d];
   }
@@ -228,11 +234,12 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(const __grid_co
 #pragma unroll
     for (int w = 0; w < kPrepThreads / 32; ++w) s += ssum[tid][w];
     // prefix[c + 1]; the block's first CTA also writes prefix[0] = 0
-    double* pre = L.bsum + (int64_t)b * 18;
+    double* pre = L.bsum + ((int64_t)b * NB + tok) * 18;
     pre[(c + 1) * 2 + tid] = nonfinite ? __longlong_as_double(0x7FF8000000000000LL) : (double)s;
     if (c == 0) pre[tid] = 0.0;
-    if (tid == 0 && c == 0) L.bexp[b] = E;
+    if (tid == 0 && c == 0) L.bexp[(int64_t)b * NB + tok] = E;
   }
+  }  // tokens
 }
 
 // ---------------------------------------------------------------- main kernel
@@ -365,6 +372,47 @@ __device__ __forceinline__ void chunk_mma(int (&acc0)[4][4], int (&acc1)[4][4], 
   }
 }
 
+// Several tokens (NB >= 2): half a chunk -- one word pair per row, 4 positions x 2 planes
+// -- against every token's fragments of those 4 k-steps.  Each operand is shifted down so
+// that its bit sits at bit 1 of each byte (weight 2 for every position): one int32 sum
+// per (plane, token) instead of one per (plane, position), at the price of a shift per
+// operand, which the NB MMAs per operand pay for.  kFirst: the first MMA of each sum.
+template <int NB, bool kFirst>
+__device__ __forceinline__ void half_chunk_mma(int (&acc0)[NB][4], int (&acc1)[NB][4], uint32_t a0, uint32_t a1,
+                                               uint32_t b0, uint32_t b1, const uint4 (&F)[NB][2]) {
+  const uint32_t ua0 = a0 ^ (a0 << 1), ua1 = a1 ^ (a1 << 1), ub0 = b0 ^ (b0 << 1), ub1 = b1 ^ (b1 << 1);
+  const uint32_t m = 0x02020202u;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t g0a0 = (ua0 >> (2 * q)) & m, g0b0 = (ub0 >> (2 * q)) & m;
+    const uint32_t g0a1 = (ua1 >> (2 * q)) & m, g0b1 = (ub1 >> (2 * q)) & m;
+    const uint32_t g1a0 = (a0 >> (2 * q)) & m, g1b0 = (b0 >> (2 * q)) & m;
+    const uint32_t g1a1 = (a1 >> (2 * q)) & m, g1b1 = (b1 >> (2 * q)) & m;
+#pragma unroll
+    for (int t = 0; t < NB; ++t) {
+      const uint32_t fx = (q & 1) ? F[t][q >> 1].z : F[t][q >> 1].x;
+      const uint32_t fy = (q & 1) ? F[t][q >> 1].w : F[t][q >> 1].y;
+      if (kFirst && q == 0) {
+        imma_16832_first(acc0[t], g0a0, g0b0, g0a1, g0b1, fx, fy);
+        imma_16832_first(acc1[t], g1a0, g1b0, g1a1, g1b1, fx, fy);
+      } else {
+        imma_16832(acc0[t], g0a0, g0b0, g0a1, g0b1, fx, fy);
+        imma_16832(acc1[t], g1a0, g1b0, g1a1, g1b1, fx, fy);
+      }
+    }
+  }
+}
+
+// A lane's fragments of half h (word pair) of a chunk for every token; fr0 points at token 0's.
+template <int NB>
+__device__ __forceinline__ void load_half_frags(uint4 (&F)[NB][2], const uint4* fr0, int h) {
+#pragma unroll
+  for (int t = 0; t < NB; ++t) {
+    F[t][0] = __ldg(fr0 + t * 128 + 2 * h);
+    F[t][1] = __ldg(fr0 + t * 128 + 2 * h + 1);
+  }
+}
+
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
                                             uint64_t* bar) {
   asm volatile(
@@ -412,8 +460,9 @@ __device__ __forceinline__ void issue_piece(const P& p, const Piece& pc, uint32_
   }
 }
 
-template <class P>
-__global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_i8_kernel(const __grid_constant__ P p) {
+template <class P, int NB>
+__global__ void __launch_bounds__(kWarps * 32, ctas_per_sm(NB)) gemv_i8_kernel(const __grid_constant__ P p) {
+  constexpr int AQ = NB == 1 ? 4 : NB;  // int32 sums per plane: per position q (one token) or per token
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
@@ -450,7 +499,9 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_i8_kernel(const 
   Piece cur = make_piece(p, c_lo, c_hi);
   issue_piece(p, cur, slots, &bars[0], lane);
   bool prep_done = false;
-  double yr[2] = {0.0, 0.0}, yi[2] = {0.0, 0.0};  // rows g, g+8 of the current tile (tq == 0)
+  double yr[NB][2], yi[NB][2];  // per token, rows g, g+8 of the current tile (tq == 0)
+#pragma unroll
+  for (int t = 0; t < NB; ++t) yr[t][0] = yr[t][1] = yi[t][0] = yi[t][1] = 0.0;
 
   for (;;) {
     const int64_t nc = cur.gbegin + cur.len;
@@ -468,22 +519,34 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_i8_kernel(const 
     // chunk and the inputs of its combine step.
     const I8Layer& L = p.L[cur.li];
     const int blk = cur.ch >> 3;
-    const uint4* fr = L.frag + (((int64_t)blk * 8 + (cur.ch & 7)) * 32 + lane) * 4;  // 32 lanes x 64 B per chunk
-    uint4 F0[4];
+    // lane's fragments of the piece's first chunk, token 0 (tokens follow at 128 uint4, chunks at NB * 128)
+    const uint4* fr = L.frag + ((((int64_t)blk * 8 + (cur.ch & 7)) * NB) * 32 + lane) * 4;
+    constexpr int kF0 = NB == 1 ? 4 : 2;  // one token: the whole first chunk; several: its first half
+    uint4 F0[NB][kF0];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) F0[k] = __ldg(fr + k);
+    for (int tk = 0; tk < NB; ++tk)
+#pragma unroll
+      for (int k = 0; k < kF0; ++k) F0[tk][k] = __ldg(fr + tk * 128 + k);
     const int t = L.nbranch == 2 ? cur.mat >> 1 : cur.mat, br = L.nbranch == 2 ? cur.mat & 1 : 0;
     float sr = 0.0f, si = 0.0f;
-    int bexp = 0;
-    double bs_re = 0.0, bs_im = 0.0;
+    int bexp[NB];
+    double bs_re[NB], bs_im[NB];
+#pragma unroll
+    for (int tk = 0; tk < NB; ++tk) {
+      bexp[tk] = 0;
+      bs_re[tk] = bs_im[tk] = 0.0;
+    }
     if (tq == 0) {
       sr = __ldg(L.scales[br] + 2 * t);
       si = __ldg(L.scales[br] + 2 * t + 1);
-      bexp = __ldg(L.bexp + blk);
-      // exact sums of v over the piece's chunks, from the prefix sums
-      const double* pre = L.bsum + (int64_t)blk * 18 + (cur.ch & 7) * 2;
-      bs_re = __ldg(pre + 2 * cur.len) - __ldg(pre);
-      bs_im = __ldg(pre + 2 * cur.len + 1) - __ldg(pre + 1);
+#pragma unroll
+      for (int tk = 0; tk < NB; ++tk) {
+        bexp[tk] = __ldg(L.bexp + (int64_t)blk * NB + tk);
+        // exact sums of v over the piece's chunks, from the prefix sums
+        const double* pre = L.bsum + ((int64_t)blk * NB + tk) * 18 + (cur.ch & 7) * 2;
+        bs_re[tk] = __ldg(pre + 2 * cur.len) - __ldg(pre);
+        bs_im[tk] = __ldg(pre + 2 * cur.len + 1) - __ldg(pre + 1);
+      }
     }
 
     int ok = 1;
@@ -504,93 +567,128 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_i8_kernel(const 
     // Plain shared loads (ordered after the barrier wait above by its memory clobber).
     const uint8_t* sbase = smem + (slot - slots0) + tq * 16;
 
-    int acc0[4][4], acc1[4][4];  // [position q][fragment reg]: the piece's int32 sums, started by chunk 0
+    int acc0[AQ][4], acc1[AQ][4];  // the piece's int32 sums, started by chunk 0: [q or token][fragment reg]
     // Positions past K carry zero activation digits, so code bytes there (stale or not) add nothing.
-    if (cur.len == kPieceChunks && piece_by_tensor(L, cur)) {  // a whole K block: chunk c at c * 1024
-      const uint4* rowa = reinterpret_cast<const uint4*>(sbase + g * 64);
-      const uint4* rowb = rowa + 512 / 16;
-      uint4 Fc[4] = {F0[0], F0[1], F0[2], F0[3]};
+    const bool whole = cur.len == kPieceChunks && piece_by_tensor(L, cur);  // a whole K block
+    // tensor layout: chunk c at c * 1024 from chunk position p0, rows at 64; row layout: chunks at 64, rows at 512
+    const bool tens = piece_by_tensor(L, cur);
+    const int cstride = tens ? 1024 / 16 : 64 / 16, rstride = tens ? 64 : 512;
+    const uint4* rowa = reinterpret_cast<const uint4*>(sbase + (tens ? piece_p0(cur) * 1024 : 0) + g * rstride);
+    const uint4* rowb = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(rowa) + 8 * rstride);
+    if constexpr (NB == 1) {
+      const uint4(&F00)[4] = F0[0];
+      if (whole) {
+        uint4 Fc[4] = {F00[0], F00[1], F00[2], F00[3]};
 #pragma unroll
-      for (int c = 0; c < kPieceChunks; ++c) {
-        uint4 Fn[4];
-        if (c + 1 < kPieceChunks) {
+        for (int c = 0; c < kPieceChunks; ++c) {
+          uint4 Fn[4];
+          if (c + 1 < kPieceChunks) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) Fn[k] = __ldg(fr + (c + 1) * 128 + k);
+            for (int k = 0; k < 4; ++k) Fn[k] = __ldg(fr + (c + 1) * 128 + k);
+          }
+          if (c == 0)
+            chunk_mma<true>(acc0, acc1, rowa, rowb, Fc);
+          else
+            chunk_mma<false>(acc0, acc1, rowa + c * 64, rowb + c * 64, Fc);
+          if (c + 1 < kPieceChunks) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) Fc[k] = Fn[k];
+          }
         }
-        if (c == 0)
-          chunk_mma<true>(acc0, acc1, rowa, rowb, Fc);
-        else
-          chunk_mma<false>(acc0, acc1, rowa + c * 64, rowb + c * 64, Fc);
-        if (c + 1 < kPieceChunks) {
+      } else {
+        chunk_mma<true>(acc0, acc1, rowa, rowb, F00);
+#pragma unroll 1
+        for (int c = 1; c < cur.len; ++c) {
+          uint4 F[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) Fc[k] = Fn[k];
+          for (int k = 0; k < 4; ++k) F[k] = __ldg(fr + c * 128 + k);
+          chunk_mma<false>(acc0, acc1, rowa + c * cstride, rowb + c * cstride, F);
         }
       }
     } else {
-      // tensor layout from chunk position p0 (strides 1024 per chunk, 64 per row) or row layout (64, 512)
-      const bool tens = piece_by_tensor(L, cur);
-      const int cstride = tens ? 1024 / 16 : 64 / 16, rstride = tens ? 64 : 512;
-      const uint4* rowa = reinterpret_cast<const uint4*>(sbase + (tens ? piece_p0(cur) * 1024 : 0) + g * rstride);
-      const uint4* rowb = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(rowa) + 8 * rstride);
-      chunk_mma<true>(acc0, acc1, rowa, rowb, F0);
-#pragma unroll 1
-      for (int c = 1; c < cur.len; ++c) {
-        uint4 F[4];
+      // half-chunks h = 2 c + word pair; each token's fragments of the next half load during this one
+      uint4 Fh[NB][2];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) F[k] = __ldg(fr + c * 128 + k);
-        chunk_mma<false>(acc0, acc1, rowa + c * cstride, rowb + c * cstride, F);
+      for (int tk = 0; tk < NB; ++tk) Fh[tk][0] = F0[tk][0], Fh[tk][1] = F0[tk][1];
+      const int nh = 2 * cur.len;
+#pragma unroll 2
+      for (int h = 0; h < nh; ++h) {
+        const int c = h >> 1, wp = h & 1;
+        uint4 Fn[NB][2];
+        if (h + 1 < nh) load_half_frags<NB>(Fn, fr + ((h + 1) >> 1) * NB * 128, (h + 1) & 1);
+        const uint4 va = rowa[c * cstride], vb = rowb[c * cstride];
+        const uint32_t a0 = wp ? va.z : va.x, a1 = wp ? va.w : va.y;
+        const uint32_t b0 = wp ? vb.z : vb.x, b1 = wp ? vb.w : vb.y;
+        if (h == 0)
+          half_chunk_mma<NB, true>(acc0, acc1, a0, a1, b0, b1, Fh);
+        else
+          half_chunk_mma<NB, false>(acc0, acc1, a0, a1, b0, b1, Fh);
+        if (h + 1 < nh) {
+#pragma unroll
+          for (int tk = 0; tk < NB; ++tk) Fh[tk][0] = Fn[tk][0], Fh[tk][1] = Fn[tk][1];
+        }
       }
     }
     __syncwarp();  // every lane is done with this slot before it is refilled
 
-    // ---- combine: both planes carry weights 2*4^q, -128 at q = 3 -> 128 G0 and 128 G1, exact int32.
-    // The digit columns are then merged in float32: its rounding (2^-24 of at most
-    // 3 sum_j |v_j| per piece) stays far inside the product tolerance.
-    float qa[2], qb[2];  // rows g, g+8: this thread's two digit columns, merged
-    {
-      int G0[4], G1[4];
+    // ---- combine, per token.  One token: the planes carry weights 2*4^q (-128 at q = 3),
+    // so 64 a_0 + 16 a_1 + 4 a_2 - a_3 = 128 G; several tokens: weight 2 everywhere, so
+    // 64 a = 128 G.  Both exact in int32.  The digit columns are then merged in float32:
+    // its rounding (2^-24 of at most 3 sum_j |v_j| per piece) stays far inside the
+    // product tolerance.
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        G0[r] = 64 * acc0[0][r] + 16 * acc0[1][r] + 4 * acc0[2][r] - acc0[3][r];
-        G1[r] = 64 * acc1[0][r] + 16 * acc1[1][r] + 4 * acc1[2][r] - acc1[3][r];
+    for (int tk = 0; tk < NB; ++tk) {
+      float qa[2], qb[2];  // rows g, g+8: this thread's two digit columns, merged
+      {
+        int G0[4], G1[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          if constexpr (NB == 1) {
+            G0[r] = 64 * acc0[0][r] + 16 * acc0[1][r] + 4 * acc0[2][r] - acc0[3][r];
+            G1[r] = 64 * acc1[0][r] + 16 * acc1[1][r] + 4 * acc1[2][r] - acc1[3][r];
+          } else {
+            G0[r] = 64 * acc0[tk][r];
+            G1[r] = 64 * acc1[tk][r];
+          }
+        }
+        const float dscale = (tq & 1) ? 65536.0f : 1.0f;  // columns 2tq, 2tq+1 hold digits 2(tq&1), +1
+        qa[0] = dscale * fmaf(256.0f, (float)G0[1], (float)G0[0]);
+        qa[1] = dscale * fmaf(256.0f, (float)G0[3], (float)G0[2]);
+        qb[0] = dscale * fmaf(256.0f, (float)G1[1], (float)G1[0]);
+        qb[1] = dscale * fmaf(256.0f, (float)G1[3], (float)G1[2]);
       }
-      const float dscale = (tq & 1) ? 65536.0f : 1.0f;  // columns 2tq, 2tq+1 hold digits 2(tq&1), +1
-      qa[0] = dscale * fmaf(256.0f, (float)G0[1], (float)G0[0]);
-      qa[1] = dscale * fmaf(256.0f, (float)G0[3], (float)G0[2]);
-      qb[0] = dscale * fmaf(256.0f, (float)G1[1], (float)G1[0]);
-      qb[1] = dscale * fmaf(256.0f, (float)G1[3], (float)G1[2]);
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      qa[r] += __shfl_xor_sync(0xffffffffu, qa[r], 1);
-      qb[r] += __shfl_xor_sync(0xffffffffu, qb[r], 1);
-    }
-    float oa[2], ob[2];  // threads tq 0,1 hold plane re, 2,3 plane im: fetch the other plane
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      oa[r] = __shfl_xor_sync(0xffffffffu, qa[r], 2);
-      ob[r] = __shfl_xor_sync(0xffffffffu, qb[r], 2);
-    }
-    if (tq == 0) {
-      const double inv = __longlong_as_double((long long)(1023 - bexp) << 52);  // 2^-E (outside float range)
-      const float fre = (float)bs_re, fim = (float)bs_im;
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
-        // G0 = QA / 128, G1 = QB / 128;  P_r = S - G0 - G1,  P_i = G0 - G1 (S: the piece's sums of v)
-        const float Prr = fre - (qa[r] + qb[r]) * 0.0078125f;
-        const float Pir = (qa[r] - qb[r]) * 0.0078125f;
-        const float Pri = fim - (oa[r] + ob[r]) * 0.0078125f;
-        const float Pii = (oa[r] - ob[r]) * 0.0078125f;
-        float vr, vi;
-        if (br == 0) {
-          vr = sr * Prr - si * Pii;
-          vi = sr * Pri + si * Pir;
-        } else {
-          vr = sr * Prr + si * Pii;
-          vi = si * Pir - sr * Pri;
+        qa[r] += __shfl_xor_sync(0xffffffffu, qa[r], 1);
+        qb[r] += __shfl_xor_sync(0xffffffffu, qb[r], 1);
+      }
+      float oa[2], ob[2];  // threads tq 0,1 hold plane re, 2,3 plane im: fetch the other plane
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        oa[r] = __shfl_xor_sync(0xffffffffu, qa[r], 2);
+        ob[r] = __shfl_xor_sync(0xffffffffu, qb[r], 2);
+      }
+      if (tq == 0) {
+        const double inv = __longlong_as_double((long long)(1023 - bexp[tk]) << 52);  // 2^-E (outside float range)
+        const float fre = (float)bs_re[tk], fim = (float)bs_im[tk];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          // G0 = QA / 128, G1 = QB / 128;  P_r = S - G0 - G1,  P_i = G0 - G1 (S: the piece's sums of v)
+          const float Prr = fre - (qa[r] + qb[r]) * 0.0078125f;
+          const float Pir = (qa[r] - qb[r]) * 0.0078125f;
+          const float Pri = fim - (oa[r] + ob[r]) * 0.0078125f;
+          const float Pii = (oa[r] - ob[r]) * 0.0078125f;
+          float vr, vi;
+          if (br == 0) {
+            vr = sr * Prr - si * Pii;
+            vi = sr * Pri + si * Pir;
+          } else {
+            vr = sr * Prr + si * Pii;
+            vi = si * Pir - sr * Pri;
+          }
+          yr[tk][r] += (double)vr * inv;
+          yi[tk][r] += (double)vi * inv;
         }
-        yr[r] += (double)vr * inv;
-        yi[r] += (double)vi * inv;
       }
     }
 
@@ -609,18 +707,23 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_i8_kernel(const 
       if (c0 == 0 && c1 == tc) {
         if (tq == 0) {
 #pragma unroll
-          for (int r = 0; r < 2; ++r)
-            if (row0 + g + 8 * r < L.N) store_y(L, row0 + g + 8 * r, (float)yr[r], (float)yi[r]);
+          for (int tk = 0; tk < NB; ++tk)
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+              if (tk < p.B && row0 + g + 8 * r < L.N)
+                store_y(L, tk * L.N + row0 + g + 8 * r, (float)yr[tk][r], (float)yi[tk][r]);
         }
       } else {
         const int64_t slot0 = cur.tile * tc;
-        float* part = L.partials + (slot0 + c0) * 32;
+        float* part = L.partials + (slot0 + c0) * 32 * NB;  // [token][row][re, im]
         if (tq == 0) {
 #pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            part[2 * (g + 8 * r)] = (float)yr[r];
-            part[2 * (g + 8 * r) + 1] = (float)yi[r];
-          }
+          for (int tk = 0; tk < NB; ++tk)
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              part[tk * 32 + 2 * (g + 8 * r)] = (float)yr[tk][r];
+              part[tk * 32 + 2 * (g + 8 * r) + 1] = (float)yi[tk][r];
+            }
         }
         if (lane == 0) L.next[slot0 + c0] = (int)c1;
         __syncwarp();
@@ -633,22 +736,30 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_i8_kernel(const 
         if ((int64_t)prev + (c1 - c0) == tc) {
           __syncwarp();
           if (lane < 16 && row0 + lane < L.N) {
-            float ar = 0.0f, ai = 0.0f;
+            float ar[NB], ai[NB];
+#pragma unroll
+            for (int tk = 0; tk < NB; ++tk) ar[tk] = ai[tk] = 0.0f;
             int64_t c = 0;
             for (int64_t guard = 0; c < tc && guard < tc; ++guard) {
-              const float* pt = L.partials + (slot0 + c) * 32 + 2 * lane;
-              ar += __ldcg(pt);
-              ai += __ldcg(pt + 1);
+              const float* pt = L.partials + (slot0 + c) * 32 * NB + 2 * lane;
+#pragma unroll
+              for (int tk = 0; tk < NB; ++tk) {
+                ar[tk] += __ldcg(pt + tk * 32);
+                ai[tk] += __ldcg(pt + tk * 32 + 1);
+              }
               const int64_t cn = __ldcg(L.next + slot0 + c);
               if (cn <= c) break;  // cannot happen: portions are non-empty and ordered
               c = cn;
             }
-            store_y(L, row0 + lane, ar, ai);
+#pragma unroll
+            for (int tk = 0; tk < NB; ++tk)
+              if (tk < p.B) store_y(L, tk * L.N + row0 + lane, ar[tk], ai[tk]);
           }
           if (lane == 0) L.tickets[cur.tile] = 0u;
         }
       }
-      yr[0] = yr[1] = yi[0] = yi[1] = 0.0;
+#pragma unroll
+      for (int tk = 0; tk < NB; ++tk) yr[tk][0] = yr[tk][1] = yi[tk][0] = yi[tk][1] = 0.0;
     }
     if (!has_next) break;
     cur = nxt;
@@ -665,7 +776,8 @@ struct WsLayout {
 
 inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-size_t layout_layers(const ifq_layer* Ls, int count, int T, WsLayout* out) {
+// nb: tokens the kernels are built for (1, 2 or 4).
+size_t layout_layers(const ifq_layer* Ls, int count, int T, int nb, WsLayout* out) {
   size_t off = 256;
   for (int i = 0; i < count; ++i) {
     const int64_t tiles = (Ls[i].N + 15) / 16;
@@ -673,14 +785,14 @@ size_t layout_layers(const ifq_layer* Ls, int count, int T, WsLayout* out) {
     const int64_t nmat = (int64_t)T * (Ls[i].codes_w ? 2 : 1);
     WsLayout w;
     w.frag = off;
-    off = align256(off + (size_t)blocks * 8 * 32 * 64);
+    off = align256(off + (size_t)blocks * 8 * nb * 32 * 64);
     w.bsum = off;
-    off = align256(off + (size_t)blocks * 18 * 8);
+    off = align256(off + (size_t)blocks * nb * 18 * 8);
     w.bexp = off;
-    off = align256(off + (size_t)blocks * 4);
+    off = align256(off + (size_t)blocks * nb * 4);
     const int64_t nch = (Ls[i].K + 255) / 256;
     w.part = off;
-    off = align256(off + (size_t)tiles * nmat * nch * 32 * 4);
+    off = align256(off + (size_t)tiles * nmat * nch * nb * 32 * 4);
     w.next = off;
     off = align256(off + (size_t)tiles * nmat * nch * 4);
     w.tick = off;
@@ -692,26 +804,32 @@ size_t layout_layers(const ifq_layer* Ls, int count, int T, WsLayout* out) {
 
 }  // namespace
 
-size_t gemv_i8_workspace_bytes(const ifq_layer* Ls, int count, int T) { return layout_layers(Ls, count, T, nullptr); }
+// Tokens per launch the integer path is built for: B = 1, 2, or 3..4 (padded with zero tokens).
+int gemv_i8_tokens(int B) { return B <= 1 ? 1 : (B == 2 ? 2 : 4); }
+
+size_t gemv_i8_workspace_bytes(const ifq_layer* Ls, int count, int T, int B) {
+  return layout_layers(Ls, count, T, gemv_i8_tokens(B), nullptr);
+}
 
 namespace {
 
-template <int kCap>
-cudaError_t launch_cap(const ifq_layer* Ls, int count, int T, void* ws, uint32_t* dev_status, cudaStream_t s) {
+template <int kCap, int NB>
+cudaError_t launch_cap(const ifq_layer* Ls, int count, int T, int B, void* ws, uint32_t* dev_status, cudaStream_t s) {
   using P = I8Params<kCap>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(gemv_i8_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMainSmem);
+    attr_err = cudaFuncSetAttribute(gemv_i8_kernel<P, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMainSmem);
   });
   if (attr_err != cudaSuccess) return attr_err;
   P p;
   memset(&p, 0, sizeof(p));
   p.count = count;
   p.T = T;
+  p.B = B;
   p.status = dev_status;
   WsLayout lay[IFQ_MAX_GROUP];
-  layout_layers(Ls, count, T, lay);
+  layout_layers(Ls, count, T, NB, lay);
   char* base = static_cast<char*>(ws);
   int64_t chunks = 0, preps = 0;
   for (int i = 0; i < count; ++i) {
@@ -757,17 +875,17 @@ cudaError_t launch_cap(const ifq_layer* Ls, int count, int T, void* ws, uint32_t
   p.total_chunks = chunks;
   if (chunks >= ((int64_t)1 << 40) || preps > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
 
-  gemv_prep_kernel<P><<<(unsigned)preps, kPrepThreads, 0, s>>>(p);
+  gemv_prep_kernel<P, NB><<<(unsigned)preps, kPrepThreads, 0, s>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int64_t ctas = (int64_t)sms * kCtasPerSm;
+  int64_t ctas = (int64_t)sms * ctas_per_sm(NB);
   const int64_t need = (chunks + kWarps - 1) / kWarps;  // at least one chunk per warp
   if (ctas > need) ctas = need;
-  p.sms = ctas == (int64_t)sms * kCtasPerSm ? sms : 0;
+  p.sms = ctas == (int64_t)sms * ctas_per_sm(NB) ? sms : 0;
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3((unsigned)ctas);
@@ -779,14 +897,24 @@ cudaError_t launch_cap(const ifq_layer* Ls, int count, int T, void* ws, uint32_t
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_i8_kernel<P>, p);
+  return cudaLaunchKernelEx(&cfg, gemv_i8_kernel<P, NB>, p);
 }
 
 }  // namespace
 
-cudaError_t launch_gemv_i8(const ifq_layer* Ls, int count, int T, void* ws, uint32_t* dev_status, cudaStream_t s) {
-  return count <= 8 ? launch_cap<8>(Ls, count, T, ws, dev_status, s)
-                    : launch_cap<IFQ_MAX_GROUP>(Ls, count, T, ws, dev_status, s);
+template <int NB>
+cudaError_t launch_nb(const ifq_layer* Ls, int count, int T, int B, void* ws, uint32_t* dev_status, cudaStream_t s) {
+  return count <= 8 ? launch_cap<8, NB>(Ls, count, T, B, ws, dev_status, s)
+                    : launch_cap<IFQ_MAX_GROUP, NB>(Ls, count, T, B, ws, dev_status, s);
+}
+
+cudaError_t launch_gemv_i8(const ifq_layer* Ls, int count, int T, int B, void* ws, uint32_t* dev_status,
+                           cudaStream_t s) {
+  switch (gemv_i8_tokens(B)) {
+    case 1: return launch_nb<1>(Ls, count, T, B, ws, dev_status, s);
+    case 2: return launch_nb<2>(Ls, count, T, B, ws, dev_status, s);
+    default: return launch_nb<4>(Ls, count, T, B, ws, dev_status, s);
+  }
 }
 
 }  // namespace ifq

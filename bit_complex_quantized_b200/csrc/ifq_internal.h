@@ -30,9 +30,11 @@ cudaError_t launch_dequantize(const ifq_dqtensor* t, int count, int T, cudaStrea
 
 cudaError_t launch_gemv(const ifq_layer* L, int count, int T, int B, uint32_t* dev_status, cudaStream_t s);
 
-// B = 1 integer tensor-core path (gemv_i8.cu) and its workspace size.
-size_t gemv_i8_workspace_bytes(const ifq_layer* L, int count, int T);
-cudaError_t launch_gemv_i8(const ifq_layer* L, int count, int T, void* ws, uint32_t* dev_status, cudaStream_t s);
+// Integer tensor-core path for B <= IFQ_I8_MAX_BATCH tokens (gemv_i8.cu) and its workspace size.
+constexpr int IFQ_I8_MAX_BATCH = 4;
+size_t gemv_i8_workspace_bytes(const ifq_layer* L, int count, int T, int B);
+cudaError_t launch_gemv_i8(const ifq_layer* L, int count, int T, int B, void* ws, uint32_t* dev_status,
+                           cudaStream_t s);
 
 // Tiled TMA descriptor (cuTensorMapEncodeTiled through the runtime's driver entry point; no
 // libcuda link).  strides: rank - 1 byte strides of dimensions 1.. ; zero fill out of bounds.

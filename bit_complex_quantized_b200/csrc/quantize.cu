@@ -187,11 +187,14 @@ __global__ void __launch_bounds__(kQThreads) quant_stage_kernel(const __grid_con
     wi[q][0] = vi.x; wi[q][1] = vi.y; wi[q][2] = vi.z; wi[q][3] = vi.w;
   }
   pdl_wait();  // the earlier stages' codes and scales are complete from here on
+  // They are read through L2 (ld.global.cg), not the read-only or L1 path: this grid starts
+  // while the previous stage still runs on the same SMs, and a line of the scales or codes
+  // cached there before the previous launches wrote it would be stale.
   double sr[8], si[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    sr[u] = u < PREV ? (double)__ldg(T.scales + 2 * u) : 0.0;
-    si[u] = u < PREV ? (double)__ldg(T.scales + 2 * u + 1) : 0.0;
+    sr[u] = u < PREV ? (double)__ldcg(T.scales + 2 * u) : 0.0;
+    si[u] = u < PREV ? (double)__ldcg(T.scales + 2 * u + 1) : 0.0;
   }
   uint32_t prev[kQuadsPerThread][8];
 #pragma unroll
@@ -199,7 +202,7 @@ __global__ void __launch_bounds__(kQThreads) quant_stage_kernel(const __grid_con
     const int64_t quad = quad0 + 32 * q;
 #pragma unroll
     for (int u = 0; u < 8; ++u)
-      prev[q][u] = (u < PREV && quad < T.nquads) ? __ldg(T.codes + (int64_t)u * T.nquads + quad) : 0u;
+      prev[q][u] = (u < PREV && quad < T.nquads) ? __ldcg(T.codes + (int64_t)u * T.nquads + quad) : 0u;
   }
 
   // Non-finite weights are rare: one check for all 16 entries, exact handling only then.
@@ -246,9 +249,9 @@ __global__ void __launch_bounds__(kQThreads) quant_reduce_kernel(const __grid_co
   unsigned long long c = 0;
   for (int64_t i = threadIdx.x; i < T.nblocks; i += kQThreads) {
     const QPartial* pp = T.partials + i;
-    a += pp->s_re;
-    b += pp->s_im;
-    c += pp->c_re;
+    a += __ldcg(&pp->s_re);  // through L2: written by the grid this one overlapped
+    b += __ldcg(&pp->s_im);
+    c += __ldcg(&pp->c_re);
   }
   block_sum3(a, b, c);
   if (threadIdx.x == 0) {

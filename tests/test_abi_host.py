@@ -86,7 +86,9 @@ def test_gemv_workspace_errors():
     arr = (L.Layer * 1)(good)
     need = lib.ifq_gemv_workspace_bytes(arr, 1, 2, 1)
     assert need > 0
-    assert lib.ifq_gemv_workspace_bytes(arr, 1, 2, 4) == 0     # B >= 2 needs none
+    assert lib.ifq_gemv_workspace_bytes(arr, 1, 2, 4) > need   # integer path up to B = 4, per token
+    assert lib.ifq_gemv_workspace_bytes(arr, 1, 2, 5) == 0     # B >= 5 needs none
+    assert _call_gemv([good], T=2, B=3, ws=FAKE, ws_bytes=lib.ifq_gemv_workspace_bytes(arr, 1, 2, 3) - 1) == 6
     assert _call_gemv([good], T=2, B=1, ws=None, ws_bytes=need) == 6
     assert _call_gemv([good], T=2, B=1, ws=FAKE, ws_bytes=need - 1) == 6
     assert _call_gemv([good], T=2, B=1, ws=FAKE + 8, ws_bytes=need) == 3

@@ -6,7 +6,7 @@ import torch
 import bit_complex_quantized_b200 as Q
 from bit_complex_quantized_b200 import workloads as W
 import oracle as O
-from ifq_testlib import DEV, gpu_quantize, to_dev
+from ifq_testlib import DEV, gpu_quantize, run_gemv, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -64,7 +64,7 @@ def test_dequantize_block_layer_and_forward():
     xi = torch.from_numpy(xi32).to(torch.bfloat16).to(DEV)
     d = dict(codes_u=c, scales_u=s, codes_w=None, scales_w=None, N=spec.N, K=spec.K, x_re=xr, x_im=xi,
              y_re=torch.empty((B, spec.N), device=DEV), y_im=torch.empty((B, spec.N), device=DEV))
-    Q.ifq_gemv([d], 2, B)
+    run_gemv([d], 2, B)
     Wr = torch.from_numpy(want_re).to(DEV).double()
     Wi = torch.from_numpy(want_im).to(DEV).double()
     xrd, xid = xr.double(), xi.double()
