@@ -143,102 +143,102 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(const __grid_co
   if (c * 256 >= klen) return;  // the block's last chunk lies before this one
 
   for (int tok = 0; tok < NB; ++tok) {
-  if (tok > 0) __syncthreads();  // the previous token's use of xs, smax and ssum is over
-  const bool live = tok < p.B;   // tokens past the batch are zero
-  unsigned int mx = 0;
+    if (tok > 0) __syncthreads();  // the previous token's use of xs, smax and ssum is over
+    const bool live = tok < p.B;   // tokens past the batch are zero
+    unsigned int mx = 0;
 #pragma unroll
-  for (int r = 0; r < kKBlock / (8 * kPrepThreads); ++r) {
+    for (int r = 0; r < kKBlock / (8 * kPrepThreads); ++r) {
 #pragma unroll
-    for (int pl = 0; pl < 2; ++pl) {
-      const int idx = (r * kPrepThreads + tid) * 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (idx < klen && live) v = __ldg(reinterpret_cast<const uint4*>(L.x[pl] + (int64_t)tok * L.K + k0 + idx));
-      *reinterpret_cast<uint4*>(&xs[pl][idx]) = v;
-      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+      for (int pl = 0; pl < 2; ++pl) {
+        const int idx = (r * kPrepThreads + tid) * 8;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (idx < klen && live) v = __ldg(reinterpret_cast<const uint4*>(L.x[pl] + (int64_t)tok * L.K + k0 + idx));
+        *reinterpret_cast<uint4*>(&xs[pl][idx]) = v;
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        mx = max(mx, wv[q] & 0x7FFFu);
-        mx = max(mx, (wv[q] >> 16) & 0x7FFFu);
+        for (int q = 0; q < 4; ++q) {
+          mx = max(mx, wv[q] & 0x7FFFu);
+          mx = max(mx, (wv[q] >> 16) & 0x7FFFu);
+        }
       }
     }
-  }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if (lane == 0) smax[warp] = mx;
-  __syncthreads();
-  mx = 0;
+    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) smax[warp] = mx;
+    __syncthreads();
+    mx = 0;
 #pragma unroll
-  for (int w = 0; w < kPrepThreads / 32; ++w) mx = max(mx, smax[w]);
-  const bool nonfinite = mx >= 0x7F80u;
-  int E = 0;  // max |x| * 2^E in [2^29, 2^30)
-  if (mx != 0 && !nonfinite) {
-    const uint32_t f = mx << 16;
-    const int e = (f >> 23) ? (int)(f >> 23) - 127 : (31 - __clz(f)) - 149;
-    E = 29 - e;
-  }
-  if (nonfinite && tid == 0 && c == 0) set_status(p.status, IFQ_DEV_NONFINITE);
-  const int E1 = min(E, 127);
-  const float f1 = __int_as_float((E1 + 127) << 23);
-  const float f2 = __int_as_float((E - E1 + 127) << 23);
+    for (int w = 0; w < kPrepThreads / 32; ++w) mx = max(mx, smax[w]);
+    const bool nonfinite = mx >= 0x7F80u;
+    int E = 0;  // max |x| * 2^E in [2^29, 2^30)
+    if (mx != 0 && !nonfinite) {
+      const uint32_t f = mx << 16;
+      const int e = (f >> 23) ? (int)(f >> 23) - 127 : (31 - __clz(f)) - 149;
+      E = 29 - e;
+    }
+    if (nonfinite && tid == 0 && c == 0) set_status(p.status, IFQ_DEV_NONFINITE);
+    const int E1 = min(E, 127);
+    const float f1 = __int_as_float((E1 + 127) << 23);
+    const float f2 = __int_as_float((E - E1 + 127) << 23);
 
-  // Exact sum of v over positions [0, 256 (c + 1)) of the block, per plane (prefix sums
-  // at chunk boundaries): thread t adds positions t, t + 128, ... below the bound.
-  long long vsum = 0;
-  {
-    const int pl = tid & 1;
-    const int bound = (c + 1) * 256 < klen ? (c + 1) * 256 : klen;
+    // Exact sum of v over positions [0, 256 (c + 1)) of the block, per plane (prefix sums
+    // at chunk boundaries): thread t adds positions t, t + 128, ... below the bound.
+    long long vsum = 0;
+    {
+      const int pl = tid & 1;
+      const int bound = (c + 1) * 256 < klen ? (c + 1) * 256 : klen;
 #pragma unroll
-    for (int r = 0; r < kKBlock / (kPrepThreads / 2); ++r) {  // independent terms: unrolled for latency
-      const int j = (tid >> 1) + r * (kPrepThreads / 2);
-      if (j < bound && !nonfinite) {
-        const float xf = __uint_as_float((uint32_t)xs[pl][j] << 16);
-        vsum += __float2int_rn((xf * f1) * f2);
+      for (int r = 0; r < kKBlock / (kPrepThreads / 2); ++r) {  // independent terms: unrolled for latency
+        const int j = (tid >> 1) + r * (kPrepThreads / 2);
+        if (j < bound && !nonfinite) {
+          const float xf = __uint_as_float((uint32_t)xs[pl][j] << 16);
+          vsum += __float2int_rn((xf * f1) * f2);
+        }
       }
     }
-  }
-  // Item (plane pl, in-byte position q, 16-position group grp = (chunk c, slice tq, word w))
-  // covers positions grp*16 + 4i + q, i = 0..3: bytes i of the code word w at position q.
-  // One item per thread: the chunk's 128 items.
-  {
-    const int it = tid;
-    const int pl = it & 1, q = (it >> 1) & 3, grp = c * 16 + (it >> 3);
-    uint32_t D[4];
+    // Item (plane pl, in-byte position q, 16-position group grp = (chunk c, slice tq, word w))
+    // covers positions grp*16 + 4i + q, i = 0..3: bytes i of the code word w at position q.
+    // One item per thread: the chunk's 128 items.
+    {
+      const int it = tid;
+      const int pl = it & 1, q = (it >> 1) & 3, grp = c * 16 + (it >> 3);
+      uint32_t D[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int j = grp * 16 + 4 * i + q;
-      int v = 0;
-      if (j < klen && !nonfinite) {
-        const float xf = __uint_as_float((uint32_t)xs[pl][j] << 16);
-        v = __float2int_rn((xf * f1) * f2);
+      for (int i = 0; i < 4; ++i) {
+        const int j = grp * 16 + 4 * i + q;
+        int v = 0;
+        if (j < klen && !nonfinite) {
+          const float xf = __uint_as_float((uint32_t)xs[pl][j] << 16);
+          v = __float2int_rn((xf * f1) * f2);
+        }
+        D[i] = ((uint32_t)v + 0x80808080u) ^ 0x80808080u;
       }
-      D[i] = ((uint32_t)v + 0x80808080u) ^ 0x80808080u;
+      const uint32_t lo01 = __byte_perm(D[0], D[1], 0x5140), lo23 = __byte_perm(D[2], D[3], 0x5140);
+      const uint32_t hi01 = __byte_perm(D[0], D[1], 0x7362), hi23 = __byte_perm(D[2], D[3], 0x7362);
+      const uint32_t dig[4] = {__byte_perm(lo01, lo23, 0x5410), __byte_perm(lo01, lo23, 0x7632),
+                               __byte_perm(hi01, hi23, 0x5410), __byte_perm(hi01, hi23, 0x7632)};
+      const int tqs = (grp >> 2) & 3, w = grp & 3;
+      const int ks = (w >> 1) * 4 + q;  // k-step within the chunk: (word pair, position)
+      // a lane's fragments for chunk c: 8 k-steps x (b0, b1) = 64 contiguous bytes
+      uint32_t* fr =
+          reinterpret_cast<uint32_t*>(L.frag + (((int64_t)b * 8 + c) * NB + tok) * 32 * 4) + ks * 2 + (w & 1);
+#pragma unroll
+      for (int d = 0; d < 4; ++d) fr[((pl * 4 + d) * 4 + tqs) * 16] = dig[d];
     }
-    const uint32_t lo01 = __byte_perm(D[0], D[1], 0x5140), lo23 = __byte_perm(D[2], D[3], 0x5140);
-    const uint32_t hi01 = __byte_perm(D[0], D[1], 0x7362), hi23 = __byte_perm(D[2], D[3], 0x7362);
-    const uint32_t dig[4] = {__byte_perm(lo01, lo23, 0x5410), __byte_perm(lo01, lo23, 0x7632),
-                             __byte_perm(hi01, hi23, 0x5410), __byte_perm(hi01, hi23, 0x7632)};
-    const int tqs = (grp >> 2) & 3, w = grp & 3;
-    const int ks = (w >> 1) * 4 + q;  // k-step within the chunk: (word pair, position)
-    // a lane's fragments for chunk c: 8 k-steps x (b0, b1) = 64 contiguous bytes
-    uint32_t* fr =
-        reinterpret_cast<uint32_t*>(L.frag + (((int64_t)b * 8 + c) * NB + tok) * 32 * 4) + ks * 2 + (w & 1);
 #pragma unroll
-    for (int d = 0; d < 4; ++d) fr[((pl * 4 + d) * 4 + tqs) * 16] = dig[d];
-  }
+    for (int o = 16; o > 1; o >>= 1) vsum += __shfl_xor_sync(0xffffffffu, vsum, o);  // even / odd lanes
+    if (lane < 2) ssum[lane][warp] = vsum;
+    __syncthreads();
+    if (tid < 2) {
+      long long s = 0;
 #pragma unroll
-  for (int o = 16; o > 1; o >>= 1) vsum += __shfl_xor_sync(0xffffffffu, vsum, o);  // even / odd lanes
-  if (lane < 2) ssum[lane][warp] = vsum;
-  __syncthreads();
-  if (tid < 2) {
-    long long s = 0;
-#pragma unroll
-    for (int w = 0; w < kPrepThreads / 32; ++w) s += ssum[tid][w];
-    // prefix[c + 1]; the block's first CTA also writes prefix[0] = 0
-    double* pre = L.bsum + ((int64_t)b * NB + tok) * 18;
-    pre[(c + 1) * 2 + tid] = nonfinite ? __longlong_as_double(0x7FF8000000000000LL) : (double)s;
-    if (c == 0) pre[tid] = 0.0;
-    if (tid == 0 && c == 0) L.bexp[(int64_t)b * NB + tok] = E;
-  }
+      for (int w = 0; w < kPrepThreads / 32; ++w) s += ssum[tid][w];
+      // prefix[c + 1]; the block's first CTA also writes prefix[0] = 0
+      double* pre = L.bsum + ((int64_t)b * NB + tok) * 18;
+      pre[(c + 1) * 2 + tid] = nonfinite ? __longlong_as_double(0x7FF8000000000000LL) : (double)s;
+      if (c == 0) pre[tid] = 0.0;
+      if (tid == 0 && c == 0) L.bexp[(int64_t)b * NB + tok] = E;
+    }
   }  // tokens
 }
 
