@@ -43,7 +43,6 @@ namespace ifq {
 namespace {
 
 constexpr int kKBlock = 2048;                  // K positions per exponent block
-constexpr int kKsteps = kKBlock / 32;          // MMA k-steps per block (64)
 constexpr int kWarps = 4;                      // warps per CTA in the main kernel
 constexpr int kPieceChunks = 8;                // at most 8 chunks (256 K positions each) per piece: one K block
 constexpr int kSlotBytes = 8192;               // one slot: 16 rows x 8 chunks x 64 bytes
@@ -408,8 +407,8 @@ template <int NB>
 __device__ __forceinline__ void load_half_frags(uint4 (&F)[NB][2], const uint4* fr0, int h) {
 #pragma unroll
   for (int t = 0; t < NB; ++t) {
-    F[t][0] = __ldg(fr0 + t * 128 + 2 * h);
-    F[t][1] = __ldg(fr0 + t * 128 + 2 * h + 1);
+    F[t][0] = fr0[t * 128 + 2 * h];
+    F[t][1] = fr0[t * 128 + 2 * h + 1];
   }
 }
 
@@ -519,14 +518,16 @@ __global__ void __launch_bounds__(kWarps * 32, ctas_per_sm(NB)) gemv_i8_kernel(c
     // chunk and the inputs of its combine step.
     const I8Layer& L = p.L[cur.li];
     const int blk = cur.ch >> 3;
-    // lane's fragments of the piece's first chunk, token 0 (tokens follow at 128 uint4, chunks at NB * 128)
+    // lane's fragments of the piece's first chunk, token 0 (tokens follow at 128 uint4, chunks at NB * 128).
+    // The prep kernel writes them while this grid runs (programmatic launch), so they are read with
+    // ordinary loads, not through the read-only path.
     const uint4* fr = L.frag + ((((int64_t)blk * 8 + (cur.ch & 7)) * NB) * 32 + lane) * 4;
     constexpr int kF0 = NB == 1 ? 4 : 2;  // one token: the whole first chunk; several: its first half
     uint4 F0[NB][kF0];
 #pragma unroll
     for (int tk = 0; tk < NB; ++tk)
 #pragma unroll
-      for (int k = 0; k < kF0; ++k) F0[tk][k] = __ldg(fr + tk * 128 + k);
+      for (int k = 0; k < kF0; ++k) F0[tk][k] = fr[tk * 128 + k];
     const int t = L.nbranch == 2 ? cur.mat >> 1 : cur.mat, br = L.nbranch == 2 ? cur.mat & 1 : 0;
     float sr = 0.0f, si = 0.0f;
     int bexp[NB];
@@ -541,11 +542,11 @@ __global__ void __launch_bounds__(kWarps * 32, ctas_per_sm(NB)) gemv_i8_kernel(c
       si = __ldg(L.scales[br] + 2 * t + 1);
 #pragma unroll
       for (int tk = 0; tk < NB; ++tk) {
-        bexp[tk] = __ldg(L.bexp + (int64_t)blk * NB + tk);
+        bexp[tk] = L.bexp[(int64_t)blk * NB + tk];
         // exact sums of v over the piece's chunks, from the prefix sums
         const double* pre = L.bsum + ((int64_t)blk * NB + tk) * 18 + (cur.ch & 7) * 2;
-        bs_re[tk] = __ldg(pre + 2 * cur.len) - __ldg(pre);
-        bs_im[tk] = __ldg(pre + 2 * cur.len + 1) - __ldg(pre + 1);
+        bs_re[tk] = pre[2 * cur.len] - pre[0];
+        bs_im[tk] = pre[2 * cur.len + 1] - pre[1];
       }
     }
 
@@ -584,7 +585,7 @@ __global__ void __launch_bounds__(kWarps * 32, ctas_per_sm(NB)) gemv_i8_kernel(c
           uint4 Fn[4];
           if (c + 1 < kPieceChunks) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) Fn[k] = __ldg(fr + (c + 1) * 128 + k);
+            for (int k = 0; k < 4; ++k) Fn[k] = fr[(c + 1) * 128 + k];
           }
           if (c == 0)
             chunk_mma<true>(acc0, acc1, rowa, rowb, Fc);
@@ -601,7 +602,7 @@ __global__ void __launch_bounds__(kWarps * 32, ctas_per_sm(NB)) gemv_i8_kernel(c
         for (int c = 1; c < cur.len; ++c) {
           uint4 F[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) F[k] = __ldg(fr + c * 128 + k);
+          for (int k = 0; k < 4; ++k) F[k] = fr[c * 128 + k];
           chunk_mma<false>(acc0, acc1, rowa + c * cstride, rowb + c * cstride, F);
         }
       }
