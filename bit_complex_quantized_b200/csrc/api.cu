@@ -181,7 +181,8 @@ ifq_status ifq_dequantize(const ifq_dqtensor* tensors, int count, int T, ifq_str
 
 size_t ifq_gemv_workspace_bytes(const ifq_layer* layers, int count, int T, int B) {
   if (check_layers(layers, count, T) != IFQ_OK || B < 1 || B > IFQ_MAX_GEMV_BATCH) return 0;
-  return B <= ifq::IFQ_I8_MAX_BATCH ? ifq::gemv_i8_workspace_bytes(layers, count, T, B) : 0;
+  return B <= ifq::IFQ_I8_MAX_BATCH ? ifq::gemv_i8_workspace_bytes(layers, count, T, B)
+                                    : ifq::gemv_bf16_workspace_bytes(layers, count, B);
 }
 
 ifq_status ifq_gemv(const ifq_layer* layers, int count, int T, int B, void* workspace, size_t workspace_bytes,
@@ -190,14 +191,15 @@ ifq_status ifq_gemv(const ifq_layer* layers, int count, int T, int B, void* work
   if (st != IFQ_OK) return st;
   if (B < 1 || B > IFQ_MAX_GEMV_BATCH) return IFQ_ERR_BATCH;
   const bool integer = B <= ifq::IFQ_I8_MAX_BATCH;
-  const size_t need = integer ? ifq::gemv_i8_workspace_bytes(layers, count, T, B) : 0;
+  const size_t need = integer ? ifq::gemv_i8_workspace_bytes(layers, count, T, B)
+                              : ifq::gemv_bf16_workspace_bytes(layers, count, B);
   if (need > 0 && (!workspace || workspace_bytes < need)) return IFQ_ERR_WORKSPACE;
   if (need > 0 && !aligned16(workspace)) return IFQ_ERR_ALIGN;
   st = check_device();
   if (st != IFQ_OK) return st;
   if (integer)
     return from_cuda(ifq::launch_gemv_i8(layers, count, T, B, workspace, dev_status, as_stream(stream)));
-  return from_cuda(ifq::launch_gemv(layers, count, T, B, dev_status, as_stream(stream)));
+  return from_cuda(ifq::launch_gemv(layers, count, T, B, workspace, dev_status, as_stream(stream)));
 }
 
 ifq_status ifq_gemm(const ifq_layer* layers, int count, int T, int64_t M, uint32_t* dev_status,

@@ -1,8 +1,12 @@
 // Decode product y = sum_t (U_hat_t x + W_hat_t conj(x)) for B = 2..16 tokens
 // ("Fairy2i write-up" §2.1, §4.2; "iFairy article" §二.2; "iFairy talk notes" §2.3.1).
 //
-// Work split: one CTA of 4 warps per 64-row block of one layer (warp w: rows
-// 16w..16w+15); blocks of longer layers are numbered first so they start first.
+// Work split: one CTA of 4 warps per (64-row block, K segment) of one layer
+// (warp w: rows 16w..16w+15).  Layers longer than kKSeg positions are cut into
+// segments of at most kKSeg, so that the CTAs carry similar work and one long
+// layer does not set the kernel's length; a segmented layer's CTAs write partial
+// sums to the workspace, which gemv_segment_sum_kernel adds in segment order.
+// Blocks of longer layers are numbered first so they start first.
 // The CTA walks K in chunks of 256 positions: the chunk of x for all B tokens
 // (both planes, bf16) is staged once in shared memory, and every warp uses it
 // for its 16 rows and every (stage, branch) code matrix.
@@ -39,6 +43,7 @@ constexpr int kChunkCodes = 256;  // codes per row per chunk: 4 threads x 16 byt
 // segments of a row, and the two planes, then fall on distinct banks.
 constexpr int kSeg = 64 + 8;
 constexpr int kXRow = 4 * kSeg;
+constexpr int kKSeg = 2048;  // K positions per CTA at most (a multiple of the 256-position chunk)
 
 struct GemvLayerArg {
   const uint8_t* codes[2];
@@ -46,11 +51,12 @@ struct GemvLayerArg {
   const uint16_t* x[2];  // re, im
   float* y[2];           // re, im
   const float* rot[2];   // optional epilogue rotation [B][N] (re, im), or null
+  float* part;           // nseg > 1: partial sums [nseg][B][N][2], else null
   int64_t N;
   int64_t K;
   int64_t block_begin;
   int nbranch;
-  int pad;
+  int nseg;              // K segments (CTAs per 64-row block)
 };
 
 struct GemvParams {
@@ -95,6 +101,7 @@ __device__ __forceinline__ void store_y(const GemvLayerArg& L, int64_t idx, floa
 // NT: MMA n-tiles (8 columns = 4 tokens each); MI: code matrices per pass over a chunk.
 template <int NT, int MI>
 __global__ void __launch_bounds__(32 * kWarps) gemv_kernel(const __grid_constant__ GemvParams p) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the segment sums may launch
   __shared__ __align__(16) uint16_t xs[4 * NT][2][kXRow];  // [token][plane][position in chunk]
   const int64_t blk = blockIdx.x;
   int oi = 0;
@@ -102,20 +109,24 @@ __global__ void __launch_bounds__(32 * kWarps) gemv_kernel(const __grid_constant
   const GemvLayerArg& L = p.L[p.order[oi]];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
-  const int64_t row0 = (blk - L.block_begin) * kRowsPerBlock + 16 * warp;
+  const int64_t lb = blk - L.block_begin;                 // (row block, segment), segment fastest
+  const int seg = (int)(lb % L.nseg);
+  const int64_t row0 = (lb / L.nseg) * kRowsPerBlock + 16 * warp;
   const int64_t rowA = row0 + g, rowB = row0 + g + 8;
   const bool okA = rowA < L.N, okB = rowB < L.N;
   const int64_t K = L.K;
   const int64_t rb = K >> 2;  // bytes per code row
   const int nmat = p.T * L.nbranch;
-  const int nchunks = (int)((K + kChunkCodes - 1) / kChunkCodes);
+  const int c_begin = seg * (kKSeg / kChunkCodes);  // this CTA's chunks of the row
+  const int nchunks_row = (int)((K + kChunkCodes - 1) / kChunkCodes);
+  const int nchunks = min(nchunks_row, c_begin + kKSeg / kChunkCodes);
   const int ntok = 4 * NT;
 
   float yr[NT][2], yi[NT][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) yr[nt][0] = yr[nt][1] = yi[nt][0] = yi[nt][1] = 0.0f;
 
-  for (int c = 0; c < nchunks; ++c) {
+  for (int c = c_begin; c < nchunks; ++c) {
     const int64_t kc = (int64_t)c * kChunkCodes;
     const int klen = (int)(K - kc < kChunkCodes ? K - kc : kChunkCodes);  // multiple of 64
     // ---- stage x of the chunk: [token][plane][256] bf16; tokens past B and positions past K are 0
@@ -219,9 +230,39 @@ __global__ void __launch_bounds__(32 * kWarps) gemv_kernel(const __grid_constant
   for (int nt = 0; nt < NT; ++nt) {
     const int tok = nt * 4 + tq;
     if (tok < p.B) {
-      if (okA) store_y(L, (int64_t)tok * L.N + rowA, yr[nt][0], yi[nt][0]);
-      if (okB) store_y(L, (int64_t)tok * L.N + rowB, yr[nt][1], yi[nt][1]);
+      if (L.nseg == 1) {
+        if (okA) store_y(L, (int64_t)tok * L.N + rowA, yr[nt][0], yi[nt][0]);
+        if (okB) store_y(L, (int64_t)tok * L.N + rowB, yr[nt][1], yi[nt][1]);
+      } else {  // partial of this segment: [seg][tok][row][re, im]
+        float* pp = L.part + (((int64_t)seg * p.B + tok) * L.N) * 2;
+        if (okA) reinterpret_cast<float2*>(pp)[rowA] = make_float2(yr[nt][0], yi[nt][0]);
+        if (okB) reinterpret_cast<float2*>(pp)[rowB] = make_float2(yr[nt][1], yi[nt][1]);
+      }
     }
+  }
+}
+
+// Segmented layers: y[tok][n] = sum over segments in order of the partials, times the
+// optional rotation.  One thread per (layer, token, output); runs after the product
+// kernel (programmatic dependent launch).
+__global__ void __launch_bounds__(256) gemv_segment_sum_kernel(const __grid_constant__ GemvParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  int64_t idx = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  for (int i = 0; i < p.count; ++i) {
+    const GemvLayerArg& L = p.L[i];
+    if (L.nseg == 1) continue;
+    const int64_t n_out = (int64_t)p.B * L.N;
+    if (idx < n_out) {
+      float ar = 0.0f, ai = 0.0f;
+      for (int sg = 0; sg < L.nseg; ++sg) {
+        const float2 v = __ldcg(reinterpret_cast<const float2*>(L.part) + (int64_t)sg * n_out + idx);
+        ar += v.x;
+        ai += v.y;
+      }
+      store_y(L, idx, ar, ai);
+      return;
+    }
+    idx -= n_out;
   }
 }
 
@@ -231,9 +272,22 @@ cudaError_t launch_nt_mi(const GemvParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+int segments_of(int64_t K) { return (int)((K + kKSeg - 1) / kKSeg); }
+
 }  // namespace
 
-cudaError_t launch_gemv(const ifq_layer* Ls, int count, int T, int B, uint32_t* dev_status, cudaStream_t s) {
+// Partial sums of the segmented layers: [nseg][B][N][2] floats each, 256-byte aligned.
+size_t gemv_bf16_workspace_bytes(const ifq_layer* Ls, int count, int B) {
+  size_t off = 0;
+  for (int i = 0; i < count; ++i) {
+    const int nseg = segments_of(Ls[i].K);
+    if (nseg > 1) off += ((size_t)nseg * B * Ls[i].N * 8 + 255) / 256 * 256;
+  }
+  return off;
+}
+
+cudaError_t launch_gemv(const ifq_layer* Ls, int count, int T, int B, void* ws, uint32_t* dev_status,
+                        cudaStream_t s) {
   GemvParams p;
   memset(&p, 0, sizeof(p));
   p.count = count;
@@ -255,7 +309,20 @@ cudaError_t launch_gemv(const ifq_layer* Ls, int count, int T, int B, uint32_t* 
     a.rot[1] = Ls[i].rot_im;
     a.N = Ls[i].N;
     a.K = Ls[i].K;
+    a.nseg = segments_of(a.K);
     p.order[i] = i;
+  }
+  int64_t sum_outputs = 0;
+  {
+    char* base = static_cast<char*>(ws);
+    size_t off = 0;
+    for (int i = 0; i < count; ++i) {
+      GemvLayerArg& a = p.L[i];
+      if (a.nseg == 1) continue;
+      a.part = reinterpret_cast<float*>(base + off);
+      off += ((size_t)a.nseg * B * a.N * 8 + 255) / 256 * 256;
+      sum_outputs += (int64_t)B * a.N;
+    }
   }
   // Longest rows first (stable): their blocks are launched first.
   for (int i = 1; i < count; ++i)
@@ -268,17 +335,30 @@ cudaError_t launch_gemv(const ifq_layer* Ls, int count, int T, int B, uint32_t* 
   for (int i = 0; i < count; ++i) {
     GemvLayerArg& a = p.L[p.order[i]];
     a.block_begin = blocks;
-    blocks += (a.N + kRowsPerBlock - 1) / kRowsPerBlock;
+    blocks += (a.N + kRowsPerBlock - 1) / kRowsPerBlock * a.nseg;
   }
   p.total_blocks = blocks;
-  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  if (blocks > 0x7fffffffLL || sum_outputs > ((int64_t)1 << 38)) return cudaErrorInvalidConfiguration;
   const int NT = (2 * B + 7) / 8;
+  cudaError_t e;
   switch (NT) {
-    case 1: return launch_nt_mi<1, 4>(p, s);
-    case 2: return launch_nt_mi<2, 2>(p, s);
-    case 3: return launch_nt_mi<3, 2>(p, s);
-    default: return launch_nt_mi<4, 2>(p, s);
+    case 1: e = launch_nt_mi<1, 4>(p, s); break;
+    case 2: e = launch_nt_mi<2, 2>(p, s); break;
+    case 3: e = launch_nt_mi<3, 2>(p, s); break;
+    default: e = launch_nt_mi<4, 2>(p, s); break;
   }
+  if (e != cudaSuccess || sum_outputs == 0) return e;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)((sum_outputs + 255) / 256));
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemv_segment_sum_kernel, p);
 }
 
 }  // namespace ifq

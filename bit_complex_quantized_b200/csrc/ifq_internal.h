@@ -28,7 +28,11 @@ cudaError_t launch_widely_linear_quantize(const ifq_wl_layer* L, int count, int 
 // Dequantized bf16 weights for training (dequantize.cu).
 cudaError_t launch_dequantize(const ifq_dqtensor* t, int count, int T, cudaStream_t s);
 
-cudaError_t launch_gemv(const ifq_layer* L, int count, int T, int B, uint32_t* dev_status, cudaStream_t s);
+// bf16 path for B > IFQ_I8_MAX_BATCH (gemv.cu); its workspace holds the partial sums of
+// layers cut into K segments (0 bytes when no layer is).
+size_t gemv_bf16_workspace_bytes(const ifq_layer* L, int count, int B);
+cudaError_t launch_gemv(const ifq_layer* L, int count, int T, int B, void* ws, uint32_t* dev_status,
+                        cudaStream_t s);
 
 // Integer tensor-core path for B <= IFQ_I8_MAX_BATCH tokens (gemv_i8.cu) and its workspace size.
 constexpr int IFQ_I8_MAX_BATCH = 4;

@@ -296,11 +296,14 @@ typedef struct {
  *           B = 2 and B = 3..4 share each operand's extraction among the
  *           tokens (B = 3 runs as 4 with a zero token).
  *   B >= 5: codes expanded in registers to exact {-2, 0, +2} bf16 operands,
- *           float32 accumulation per axis class.
+ *           float32 accumulation per axis class; a layer longer than 2048
+ *           positions is cut into K segments whose partial sums are added in
+ *           segment order through the workspace.
  * workspace: device scratch of ifq_gemv_workspace_bytes() bytes, 16-byte
  *           aligned, owned by the caller; no initial contents needed.  Calls
  *           that share a workspace must not overlap on the GPU.  May be NULL
- *           when ifq_gemv_workspace_bytes() returns 0 (B >= 5).
+ *           when ifq_gemv_workspace_bytes() returns 0 (B >= 5 with every
+ *           K <= 2048).
  * dev_status may be NULL.  A NaN or Inf activation sets IFQ_DEV_NONFINITE
  * (B <= 4: the affected outputs are NaN); a lost pipeline wait sets
  * IFQ_DEV_TIMEOUT. */
