@@ -287,7 +287,7 @@ def oracle_decode_sample(seconds_budget=12.0, rows_per_layer=256):
 
 # ---------------------------------------------------------------- decode at B = 16
 def decode_batch(block, B, reps=20):
-    """The block's decode product at batch B (B <= 4: the integer path; B >= 5: bf16 mma.sync), after
+    """The block's decode product at batch B (B <= 2: the integer path; B >= 3: bf16 mma.sync), after
     an L2 flush, through the same grouped call; reported beside the step, not part of it."""
     layers = Q.LayerSet(block._layers(block.cfg, B))
     nws = Q.ifq_gemv_workspace_bytes(layers, block.T, B)
@@ -306,7 +306,7 @@ def decode_batch(block, B, reps=20):
     nbytes = block.gemv_bytes(B)
     gbs = nbytes / t / 1e9
     return {"B": B, "us": t * 1e6, "algorithmic_bytes": nbytes, "GBps": gbs,
-            "frac_of_hbm": gbs / float(peaks()[0]["hbm_gbs"]), "path": "integer" if B <= 4 else "bf16"}
+            "frac_of_hbm": gbs / float(peaks()[0]["hbm_gbs"]), "path": "integer" if B <= 2 else "bf16 (K segments)"}
 
 
 def decode_b16(block, reps=20):

@@ -805,8 +805,9 @@ size_t layout_layers(const ifq_layer* Ls, int count, int T, int nb, WsLayout* ou
 
 }  // namespace
 
-// Tokens per launch the integer path is built for: B = 1, 2, or 3..4 (padded with zero tokens).
-int gemv_i8_tokens(int B) { return B <= 1 ? 1 : (B == 2 ? 2 : 4); }
+// Tokens per launch the integer path is built for: B = 1 or 2.  (The template also builds
+// for four tokens, B = 3..4 padded; the bf16 path with K segments measured faster there.)
+int gemv_i8_tokens(int B) { return B <= 1 ? 1 : 2; }
 
 size_t gemv_i8_workspace_bytes(const ifq_layer* Ls, int count, int T, int B) {
   return layout_layers(Ls, count, T, gemv_i8_tokens(B), nullptr);
@@ -911,11 +912,8 @@ cudaError_t launch_nb(const ifq_layer* Ls, int count, int T, int B, void* ws, ui
 
 cudaError_t launch_gemv_i8(const ifq_layer* Ls, int count, int T, int B, void* ws, uint32_t* dev_status,
                            cudaStream_t s) {
-  switch (gemv_i8_tokens(B)) {
-    case 1: return launch_nb<1>(Ls, count, T, B, ws, dev_status, s);
-    case 2: return launch_nb<2>(Ls, count, T, B, ws, dev_status, s);
-    default: return launch_nb<4>(Ls, count, T, B, ws, dev_status, s);
-  }
+  return gemv_i8_tokens(B) == 1 ? launch_nb<1>(Ls, count, T, B, ws, dev_status, s)
+                                : launch_nb<2>(Ls, count, T, B, ws, dev_status, s);
 }
 
 }  // namespace ifq

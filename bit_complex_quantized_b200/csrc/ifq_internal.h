@@ -35,7 +35,7 @@ cudaError_t launch_gemv(const ifq_layer* L, int count, int T, int B, void* ws, u
                         cudaStream_t s);
 
 // Integer tensor-core path for B <= IFQ_I8_MAX_BATCH tokens (gemv_i8.cu) and its workspace size.
-constexpr int IFQ_I8_MAX_BATCH = 4;
+constexpr int IFQ_I8_MAX_BATCH = 2;
 size_t gemv_i8_workspace_bytes(const ifq_layer* L, int count, int T, int B);
 cudaError_t launch_gemv_i8(const ifq_layer* L, int count, int T, int B, void* ws, uint32_t* dev_status,
                            cudaStream_t s);

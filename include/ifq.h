@@ -284,7 +284,7 @@ typedef struct {
 
 /* Decode product for B = 1..IFQ_MAX_GEMV_BATCH tokens per layer; all `count`
  * layers (1..IFQ_MAX_GROUP) run in one launch.  Codes stream from HBM once.
- *   B <= 4: exact integer tensor-core path.  Each code becomes two 0/1 planes
+ *   B <= 2: exact integer tensor-core path.  Each code becomes two 0/1 planes
  *           of its Gray re-coding (g1 = sign, g0 = axis XOR sign, so that
  *           Re b = 1 - g0 - g1 and Im b = g0 - g1 are affine in the bits); the
  *           activations of each 2048-wide K block are scaled by a power of two
@@ -293,19 +293,18 @@ typedef struct {
  *           of the activation scaling (below 2^-29 of the block's largest |x|
  *           per position, per token).  Partial sums are combined in a fixed
  *           order through the workspace, so results are bit-reproducible.
- *           B = 2 and B = 3..4 share each operand's extraction among the
- *           tokens (B = 3 runs as 4 with a zero token).
- *   B >= 5: codes expanded in registers to exact {-2, 0, +2} bf16 operands,
+ *           B = 2 shares each operand's extraction between the tokens.
+ *   B >= 3: codes expanded in registers to exact {-2, 0, +2} bf16 operands,
  *           float32 accumulation per axis class; a layer longer than 2048
  *           positions is cut into K segments whose partial sums are added in
  *           segment order through the workspace.
  * workspace: device scratch of ifq_gemv_workspace_bytes() bytes, 16-byte
  *           aligned, owned by the caller; no initial contents needed.  Calls
  *           that share a workspace must not overlap on the GPU.  May be NULL
- *           when ifq_gemv_workspace_bytes() returns 0 (B >= 5 with every
+ *           when ifq_gemv_workspace_bytes() returns 0 (B >= 3 with every
  *           K <= 2048).
  * dev_status may be NULL.  A NaN or Inf activation sets IFQ_DEV_NONFINITE
- * (B <= 4: the affected outputs are NaN); a lost pipeline wait sets
+ * (B <= 2: the affected outputs are NaN); a lost pipeline wait sets
  * IFQ_DEV_TIMEOUT. */
 size_t ifq_gemv_workspace_bytes(const ifq_layer* layers, int count, int T, int B);
 

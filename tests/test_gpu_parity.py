@@ -118,7 +118,8 @@ def c3_quantized():
 def test_c3_gemv_b1_b16(c3_quantized):
     cfg, outs, host = c3_quantized
     rng = np.random.default_rng(3)
-    # the configuration's batches (1, 16) and the integer path's several-token sizes (2, 3, 4)
+    # the configuration's batches (1, 16), the integer path's two tokens and the bf16 path at 3, 4
+    # (the down projection, K = 5504, in three segments)
     for B in sorted(set(cfg.batches) | {2, 3, 4}):
         descs, xs = [], []
         for i, spec in enumerate(cfg.layers):
@@ -383,8 +384,8 @@ def test_b1_nonfinite_activation_is_flagged():
 
 def test_max_group_of_32_layers():
     """IFQ_MAX_GROUP layers in one grouped call: mixed shapes, every fourth layer with the conj
-    branch, at B = 1 and B = 3 (integer path, one and four tokens: layer changes inside warp
-    ranges) and B = 5 (bf16 path)."""
+    branch, at B = 1 and B = 2 (integer path, one and two tokens: layer changes inside warp
+    ranges) and B = 5 (bf16 path, the K = 2112 layers in two segments)."""
     rng = np.random.default_rng(3232)
     T = 2
     specs = [(16 + 8 * (i % 9), (64, 128, 256, 320, 2112)[i % 5], i % 4 == 0) for i in range(Q.IFQ_MAX_GROUP)]
@@ -399,7 +400,7 @@ def test_max_group_of_32_layers():
     host = [(c.cpu().numpy(), s.cpu().numpy()) for c, s in outs]
     for (wr, wi), (cn, sn) in zip(flat, host):
         check_quantized(wr, wi, cn, sn, T)
-    for B in (1, 3, 5):
+    for B in (1, 2, 5):
         descs, ref = [], []
         j = 0
         for (N, K, conj) in specs:
