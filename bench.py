@@ -136,8 +136,8 @@ class Block:
     """Device-resident state of the 7B-shaped block: real weights, planes, codes, activations."""
 
     def __init__(self, dev, gemm_M=2048, decode_B=1):
-        self.cfg = W.config("c3")
-        self.cfg4 = W.config("c4")
+        self.cfg = W.config("llama7b")
+        self.cfg4 = W.config("llama7b_prefill")
         self.T = self.cfg.T
         self.dev = dev
         self.R = []
@@ -241,7 +241,7 @@ def oracle_sample_layers(rows_per_layer):
     sampled rows (setup, untimed), and the block's activations."""
     import oracle as O
     from oracle import cref
-    cfg = W.config("c3")
+    cfg = W.config("llama7b")
     rng = np.random.default_rng(123)
     layers = []
     for i, spec in enumerate(cfg.layers):
@@ -565,10 +565,10 @@ def run_ours(args):
     kernels = {
         "gemv": {"bound": "hbm", "achieved": gemv_gbs, "peak": hbm, "unit": "GB/s", "frac": gemv_gbs / hbm,
                  "us": t_gemv * 1e6, "algorithmic_bytes": gemv_bytes,
-                 "traffic": recorded_traffic("gemv_i8.cu", "gemv", "c3_b1")},
+                 "traffic": recorded_traffic("gemv_i8.cu", "gemv", "llama7b_b1")},
         "gemm": {"bound": "tensor", "achieved": gemm_tops, "peak": tf_sus, "unit": "TFLOP/s",
                  "frac": gemm_tops / tf_sus, "us": t_gemm * 1e6, "equiv_flops": block.gemm_flops(),
-                 "traffic": recorded_traffic("gemm.cu", "gemm", "c4_m2048")},
+                 "traffic": recorded_traffic("gemm.cu", "gemm", "llama7b_prefill_m2048")},
         "quantize": {"bound": "hbm", "achieved": quant_gbs, "peak": hbm, "unit": "GB/s", "frac": quant_gbs / hbm,
                      "us": t_quant * 1e6, "algorithmic_bytes": block.quant_bytes()},
         "convert": {"bound": "hbm", "achieved": conv_gbs, "peak": hbm, "unit": "GB/s", "frac": conv_gbs / hbm,
@@ -647,8 +647,8 @@ def run_case(args):
     g = torch.Generator(device=dev)
     g.manual_seed(0)
     if args.case == "gemv":
-        # 7B-shaped block (c3, 50.6 MB of codes) or 70B-shaped layer set (c5, 321 MB, larger
-        # than L2), random codes: the kernel's work does not depend on code values.  The L2 is
+        # 7B-shaped block (llama7b, 50.6 MB of codes) or 70B-shaped layer set (llama70b, 321 MB,
+        # larger than L2), random codes: the kernel's work does not depend on code values.  The L2 is
         # flushed before every timed call.
         cfg = W.config(args.workload)
         layers = []
@@ -670,7 +670,7 @@ def run_case(args):
             Q.ifq_gemv(layers, cfg.T, args.batch, workspace=gws)
         label = f"gemv {args.workload} B={args.batch}"
     elif args.case == "gemm":
-        cfg = W.config("c4")
+        cfg = W.config("llama7b_prefill")
         spec = cfg.layers[4]  # gate: N = 5504, K = 2048
         M = 2048
 
@@ -685,9 +685,9 @@ def run_case(args):
 
         def fn():
             Q.ifq_gemm([L], 2, M)
-        label = "gemm c4 gate M=2048"
+        label = "gemm llama7b gate M=2048"
     elif args.case == "quant":
-        cfg = W.config("c3")
+        cfg = W.config("llama7b")
         spec = cfg.layers[4]
         ts = []
         for _ in range(2):
@@ -700,9 +700,9 @@ def run_case(args):
 
         def fn():
             Q.ifq_quantize_pack(ts, 2, wsb)
-        label = "quantize c3 gate U+W T=2"
+        label = "quantize llama7b gate U+W T=2"
     elif args.case == "wlq":
-        cfg = W.config("c3")
+        cfg = W.config("llama7b")
         spec = cfg.layers[4]
         R = 0.02 * torch.randn(spec.real_shape, device=dev, generator=g)
         f = lambda: torch.empty((spec.N, spec.K), device=dev)  # noqa: E731
@@ -714,9 +714,9 @@ def run_case(args):
 
         def fn():
             Q.ifq_widely_linear_quantize_pack(wl, 2, wsb)
-        label = "fused convert + quantize c3 gate T=2"
+        label = "fused convert + quantize llama7b gate T=2"
     elif args.case == "dequant":
-        cfg = W.config("c3")
+        cfg = W.config("llama7b")
         spec = cfg.layers[4]
         cb = torch.randint(0, 256, (2, spec.N, spec.K // 4), dtype=torch.uint8, device=dev, generator=g)
         sc = torch.full((2, 2), 0.01, device=dev)
@@ -725,9 +725,9 @@ def run_case(args):
 
         def fn():
             Q.ifq_dequantize([(cb, sc, outp[0], outp[1])], 2)
-        label = "dequantize bf16 c3 gate T=2"
+        label = "dequantize bf16 llama7b gate T=2"
     elif args.case == "convert":
-        cfg = W.config("c3")
+        cfg = W.config("llama7b")
         spec = cfg.layers[4]
         R = 0.02 * torch.randn(spec.real_shape, device=dev, generator=g)
         planes = [torch.empty((spec.N, spec.K), device=dev) for _ in range(4)]
@@ -735,7 +735,7 @@ def run_case(args):
 
         def fn():
             Q.ifq_widely_linear_from_real(R, *planes)
-        label = "convert c3 gate"
+        label = "convert llama7b gate"
     else:
         raise SystemExit("unknown case")
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -765,7 +765,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--case", choices=["gemv", "gemm", "quant", "convert", "wlq", "dequant"], default=None)
     ap.add_argument("--batch", type=int, default=1)
-    ap.add_argument("--workload", choices=["c3", "c5"], default="c5", help="layer set of --case gemv")
+    ap.add_argument("--workload", choices=["llama7b", "llama70b"], default="llama70b", help="layer set of --case gemv")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-dense", action="store_true", help="skip the cuBLAS bf16 dense comparator")

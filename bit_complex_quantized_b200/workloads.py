@@ -1,5 +1,5 @@
 """Seeded synthetic workloads: shapes, distributions and seeds of the five
-benchmark configurations.  Random numbers only -- none of the method's
+benchmark workloads.  Random numbers only -- none of the method's
 arithmetic lives here; the CUDA path and the oracle both take these arrays as
 inputs.
 
@@ -52,29 +52,35 @@ def _block(prefix_sigma, hidden_real, ffn_real, kind):
 
 
 def config(name: str) -> Config:
-    """The five configurations, by short name c1..c5."""
-    if name == "c1":   # single complex layer, 256 x 256, 1 stage, no conjugate branch
-        return Config("c1", 0, 1, False, [1], [LayerSpec("w", "complex", 256, 256, 0.02)], prefill_M=0)
-    if name == "c2":   # plain complex block, hidden 1024, FFN 2816, 1 stage
-        return Config("c2", 1, 1, False, [1, 8], _block(0.02, 1024, 2816, "complex"), prefill_M=0)
-    if name == "c3":   # LLaMA-2-7B-shaped real layers -> (U, W), 2 stages
-        return Config("c3", 2, 2, True, [1, 16], _block(0.02, 4096, 11008, "real"), prefill_M=2048)
-    if name == "c4":   # prefill on the c3 matrices, M = 2048 tokens, activation seed 3
-        c = config("c3")
-        return Config("c4", 3, 2, True, [], c.layers, prefill_M=2048)
-    if name == "c5":   # LLaMA-2-70B-shaped layer, 3 stages; k, v: 8192 in -> 1024 out
+    """The five workloads, by name:
+    layer256         one complex layer, 256 x 256, 1 stage, no conjugate branch
+    block1024        plain complex transformer block, hidden 1024, FFN 2816, 1 stage
+    llama7b          LLaMA-2-7B-shaped real block -> (U, W), 2 stages
+    llama7b_prefill  prefill on the llama7b matrices, M = 2048 tokens
+    llama70b         LLaMA-2-70B-shaped layer set -> (U, W), 3 stages
+    """
+    if name == "layer256":
+        return Config("layer256", 0, 1, False, [1], [LayerSpec("w", "complex", 256, 256, 0.02)], prefill_M=0)
+    if name == "block1024":
+        return Config("block1024", 1, 1, False, [1, 8], _block(0.02, 1024, 2816, "complex"), prefill_M=0)
+    if name == "llama7b":
+        return Config("llama7b", 2, 2, True, [1, 16], _block(0.02, 4096, 11008, "real"), prefill_M=2048)
+    if name == "llama7b_prefill":   # the llama7b weights; activation seed 3
+        c = config("llama7b")
+        return Config("llama7b_prefill", 3, 2, True, [], c.layers, prefill_M=2048)
+    if name == "llama70b":   # k, v: 8192 in -> 1024 out
         s = 0.015
         L = [LayerSpec("q", "real", 4096, 4096, s), LayerSpec("k", "real", 512, 4096, s),
              LayerSpec("v", "real", 512, 4096, s), LayerSpec("o", "real", 4096, 4096, s),
              LayerSpec("gate", "real", 14336, 4096, s), LayerSpec("up", "real", 14336, 4096, s),
              LayerSpec("down", "real", 4096, 14336, s)]
-        return Config("c5", 4, 3, True, [1, 8], L, prefill_M=0)
+        return Config("llama70b", 4, 3, True, [1, 8], L, prefill_M=0)
     raise KeyError(name)
 
 
 def weight_seed(cfg: Config, layer: int):
-    # c4 shares the c3 weights
-    return [config("c3").seed if cfg.name == "c4" else cfg.seed, 0, layer]
+    # the prefill workload shares the llama7b weights
+    return [config("llama7b").seed if cfg.name == "llama7b_prefill" else cfg.seed, 0, layer]
 
 
 def complex_weights(cfg: Config, layer: int, rows=None):

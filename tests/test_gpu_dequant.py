@@ -40,9 +40,9 @@ def test_dequantize_bit_exact(shapes, T):
 
 
 def test_dequantize_block_layer_and_forward():
-    """The c3 gate layer (5504 x 2048, T = 2): bit-exact weights, and the training forward pass
+    """The llama7b gate layer (5504 x 2048, T = 2): bit-exact weights, and the training forward pass
     x W_hat^T (a plain bf16 matmul of the planes) agrees with the quantized product."""
-    cfg = W.config("c3")
+    cfg = W.config("llama7b")
     spec = cfg.layers[4]
     rng = np.random.default_rng(9)
     wr = to_dev((0.02 * rng.standard_normal((spec.N, spec.K))).astype(np.float32))

@@ -86,7 +86,7 @@ def test_fused_equals_two_pass_and_oracle(n, m, T):
 
 def test_fused_block_of_seven_layers_equals_two_pass():
     """The LLaMA-2-7B-shaped block (seven real layers, 2 stages) in one grouped call."""
-    cfg = W.config("c3")
+    cfg = W.config("llama7b")
     Rs = [to_dev(W.real_weight(cfg, i)) for i in range(len(cfg.layers))]
     a = fused(Rs, cfg.T)
     b = two_pass(Rs, cfg.T)

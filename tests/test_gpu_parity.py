@@ -33,8 +33,8 @@ def _x(cfg, i, rows):
 
 
 # ---------------------------------------------------------------- config 1
-def test_c1_single_layer_quantize_and_gemv():
-    cfg = W.config("c1")
+def test_layer256_quantize_and_gemv():
+    cfg = W.config("layer256")
     ws_np, ws_dev = _complex_cfg_weights(cfg)
     st = status_word()
     (codes, scales), = gpu_quantize(ws_dev, cfg.T, st)
@@ -51,8 +51,8 @@ def test_c1_single_layer_quantize_and_gemv():
 
 
 # ---------------------------------------------------------------- config 2
-def test_c2_block_quantize_gemv_b1_b8_and_gemm():
-    cfg = W.config("c2")
+def test_block1024_quantize_gemv_b1_b8_and_gemm():
+    cfg = W.config("block1024")
     ws_np, ws_dev = _complex_cfg_weights(cfg)
     outs = gpu_quantize(ws_dev, cfg.T)
     torch.cuda.synchronize()
@@ -88,10 +88,10 @@ def test_c2_block_quantize_gemv_b1_b8_and_gemm():
 
 # ---------------------------------------------------------------- configs 3 and 4
 @pytest.fixture(scope="module")
-def c3_quantized():
+def llama7b_quantized():
     """Convert the seven 7B-shaped real layers, quantize all 14 U/W tensors in one
     grouped call (the config-4 batched quantizer), check conversion and codes."""
-    cfg = W.config("c3")
+    cfg = W.config("llama7b")
     planes, ws_np = [], []
     for i in range(len(cfg.layers)):
         R = W.real_weight(cfg, i)
@@ -111,12 +111,12 @@ def c3_quantized():
     mism = []
     for (wr, wi), (cn, sn) in zip(ws_dev, host):
         mism.append(check_quantized(wr.cpu().numpy(), wi.cpu().numpy(), cn, sn, cfg.T))
-    print("c3 near-boundary mismatches per tensor and stage:", mism)
+    print("llama7b near-boundary mismatches per tensor and stage:", mism)
     return cfg, outs, host
 
 
-def test_c3_gemv_b1_b16(c3_quantized):
-    cfg, outs, host = c3_quantized
+def test_llama7b_gemv_b1_b16(llama7b_quantized):
+    cfg, outs, host = llama7b_quantized
     rng = np.random.default_rng(3)
     # the configuration's batches (1, 16), the integer path's two tokens and the bf16 path at 3, 4
     # (the down projection, K = 5504, in three segments)
@@ -135,9 +135,9 @@ def test_c3_gemv_b1_b16(c3_quantized):
             check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cun, sun, cwn, swn, *xs[i], rows)
 
 
-def test_c4_gemm_m2048(c3_quantized):
-    cfg3, outs, host = c3_quantized
-    cfg = W.config("c4")
+def test_llama7b_prefill_gemm_m2048(llama7b_quantized):
+    cfg3, outs, host = llama7b_quantized
+    cfg = W.config("llama7b_prefill")
     M = cfg.prefill_M
     rng = np.random.default_rng(4)
     descs, xs = [], []
@@ -156,8 +156,8 @@ def test_c4_gemm_m2048(c3_quantized):
         check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cun, sun, cwn, swn, *xs[i], rows)
 
 
-def test_c3_gemv_and_gemm_agree_on_same_tokens(c3_quantized):
-    cfg, outs, host = c3_quantized
+def test_llama7b_gemv_and_gemm_agree_on_same_tokens(llama7b_quantized):
+    cfg, outs, host = llama7b_quantized
     i = 6  # down projection, K = 5504
     spec = cfg.layers[i]
     B = 16
@@ -176,8 +176,8 @@ def test_c3_gemv_and_gemm_agree_on_same_tokens(c3_quantized):
 
 # ---------------------------------------------------------------- config 5
 @pytest.mark.slow
-def test_c5_convert_quantize_gemv():
-    cfg = W.config("c5")
+def test_llama70b_convert_quantize_gemv():
+    cfg = W.config("llama70b")
     rng = np.random.default_rng(5)
     outs_all, host_all = [], []
     for i, spec in enumerate(cfg.layers):
