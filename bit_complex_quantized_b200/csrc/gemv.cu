@@ -1,4 +1,5 @@
-// Decode product y = sum_t (U_hat_t x + W_hat_t conj(x)) for B = 2..16 tokens
+// Decode product y = sum_t (U_hat_t x + W_hat_t conj(x)) for up to 16 tokens (the C ABI
+// sends B >= 3 here; one and two tokens take the integer path)
 // ("Fairy2i write-up" §2.1, §4.2; "iFairy article" §二.2; "iFairy talk notes" §2.3.1).
 //
 // Work split: one CTA of 4 warps per (64-row block, K segment) of one layer
