@@ -312,9 +312,10 @@ ifq_status ifq_gemv(const ifq_layer* layers, int count, int T, int B, void* work
                     uint32_t* dev_status, ifq_stream_t stream);
 
 /* Prefill product for M >= 1 tokens (meant for M >= 128) on the tensor cores:
- * codes are expanded in shared memory to exact {-2, 0, +2} bf16 operands, the
- * +-1 and +-i classes accumulate in separate float32 TMEM accumulators, and the
- * scales are applied per (stage, branch) in the epilogue.  Layers run one after
+ * codes are expanded straight into TMEM as exact {-2, 0, +2} bf16 operands (the
+ * MMA's A operand), the +-1 and +-i classes accumulate in separate rows of a
+ * float32 TMEM accumulator, and the scales are applied per (stage, branch) in
+ * the epilogue.  Layers run one after
  * another on the stream.  dev_status may be NULL (timeouts then go unreported). */
 ifq_status ifq_gemm(const ifq_layer* layers, int count, int T, int64_t M, uint32_t* dev_status,
                     ifq_stream_t stream);
