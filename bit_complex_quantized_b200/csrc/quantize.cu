@@ -518,22 +518,49 @@ cudaError_t launch_widely_linear_quantize(const ifq_wl_layer* Ls, int count, int
 // the rest of the device).  Same layout as the caller workspace above.
 static __device__ __align__(256) unsigned char g_quant_scratch[IFQ_QUANT_STATIC_SCRATCH_BYTES];
 
+// The current driver context, through the runtime's driver entry point (no libcuda link); null if
+// the entry point is unavailable.
+static void* current_context() {
+  typedef CUresult (*GetCurrentFn)(CUcontext*);
+  static GetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<GetCurrentFn>(p);
+  });
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
 cudaError_t launch_quantize_static(const ifq_qtensor* t, int count, int T, uint32_t* dev_status, cudaStream_t s) {
   constexpr int kCachedDevices = 64;
   static std::mutex mu;
   static void* addr[kCachedDevices] = {};
+  static void* ctx_of[kCachedDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  // The address is cached per device together with the context it was looked up in: after a
+  // device reset, or when the caller runs in a context other than the one cached, the array lives
+  // at a new address and is looked up again.
+  void* ctx = current_context();
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(mu);
-    if (dev >= 0 && dev < kCachedDevices) scratch = addr[dev];
+    const bool cacheable = dev >= 0 && dev < kCachedDevices && ctx != nullptr;
+    if (cacheable && ctx_of[dev] == ctx) scratch = addr[dev];
     if (!scratch) {
-      // Once per device, with that device current: the array's address in its context.
+      // With the device current: the array's address in the current context.
       e = cudaGetSymbolAddress(&scratch, g_quant_scratch);
       if (e != cudaSuccess) return e;
-      if (dev >= 0 && dev < kCachedDevices) addr[dev] = scratch;
+      if (cacheable) {
+        addr[dev] = scratch;
+        ctx_of[dev] = ctx;
+      }
     }
   }
   return launch_quantize(t, count, T, scratch, dev_status, s);

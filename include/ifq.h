@@ -149,9 +149,12 @@ ifq_status ifq_quantize_pack(const ifq_qtensor* tensors, int count, int T, void*
  * The scratch needs no initial contents: every call writes each part of it
  * before reading it.
  * The first call on a device (with that device current) looks up the array's
- * device address once (cudaGetSymbolAddress) and may load the library's device
- * code; make that first call before anything that must not see such set-up,
- * such as a stream capture.
+ * device address (cudaGetSymbolAddress) and may load the library's device code;
+ * make that first call before anything that must not see such set-up, such as
+ * a stream capture.  The address is kept per device together with the driver
+ * context it belongs to, and looked up again when a call runs in another
+ * context (a context of the caller's own, or the new primary context after a
+ * device reset).
  * There is one array per device: calls whose work may overlap on the GPU
  * (unordered streams, or several host threads) race on it and give wrong
  * results.  Order such calls on one stream.

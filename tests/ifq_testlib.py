@@ -10,6 +10,9 @@ compare with the oracle under the acceptance rules:
   * every output |y - y_ref| <= 1e-5 sum_{t,branch}(s_re + s_im) sum_j(|Re x_j| + |Im x_j|),
     with y_ref the complex128 product of the same codes, scales and bf16 x.
 """
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -121,6 +124,29 @@ def check_product(y_re, y_im, cu, su, cw, sw, x_re, x_im, rows=None, slack=1.0):
     worst = float(np.max(err / bound))
     assert np.all(err <= bound), f"max err/bound = {worst}"
     return worst
+
+
+def record(name, payload):
+    """Write a JSON record of a test's counts to $IFQ_RECORD_DIR/<name>.json when that variable is set
+    (the near-boundary mismatch counts that the acceptance rules ask to report)."""
+    d = os.environ.get("IFQ_RECORD_DIR")
+    if not d:
+        return
+    os.makedirs(d, exist_ok=True)
+    with open(os.path.join(d, name + ".json"), "w") as f:
+        json.dump(payload, f, indent=1)
+
+
+def tile_rows(N, rng, tile=64, group=16):
+    """Output columns that cover every product tile: both edges of each `tile`-wide block of
+    outputs and one random column inside each `group`-wide run of it (sorted, unique)."""
+    cols = set()
+    for t0 in range(0, N, tile):
+        t1 = min(N, t0 + tile)
+        cols.update((t0, t1 - 1))
+        for g0 in range(t0, t1, group):
+            cols.add(int(rng.integers(g0, min(t1, g0 + group))))
+    return np.array(sorted(cols))
 
 
 def sample_rows(N, k, rng):

@@ -541,3 +541,147 @@ def test_dequantize_bf16_is_within_rounding_of_the_exact_sum():
         tot = float(np.sum(sc, dtype=np.float64))
         for got, want in ((re, exact.real), (im, exact.imag)):
             assert np.all(np.abs(got - want) <= 2.0 ** -8 * np.abs(want) + 2.0 ** -20 * tot)
+
+
+# ---------------------------------------------------------------- bf16 rounding and decoding
+def _rne(q, p, emin):
+    """Exact rational q rounded to the nearest binary floating-point value with p significant bits,
+    ties to the even significand, with subnormals below 2^emin on the fixed quantum 2^(emin - p + 1).
+    Written from the definition of round-to-nearest-even; no overflow handling (returns a Fraction)."""
+    q = Fraction(q)
+    if q == 0:
+        return Fraction(0)
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    quantum = Fraction(2) ** (max(e, emin) - p + 1)
+    n = a / quantum
+    f = n.numerator // n.denominator
+    rest = n - f
+    if rest > Fraction(1, 2) or (rest == Fraction(1, 2) and f % 2 == 1):
+        f += 1
+    return (1 if q > 0 else -1) * f * quantum
+
+
+def _bf16_by_definition(x32):
+    """bf16 RNE of one finite float32 value, through exact arithmetic; +-inf past the largest finite."""
+    r = _rne(Fraction(float(x32)), 8, -126)
+    if abs(r) >= Fraction(2) ** 128:
+        return float("inf") if r > 0 else float("-inf")
+    return float(r)
+
+
+# (float32 bits, expected bf16 bits): worked by hand from round-to-nearest-even on the upper 16 bits
+BF16_HAND = [
+    (0x3F800000, 0x3F80),  # 1.0 is exact
+    (0x3F808000, 0x3F80),  # exact tie, kept LSB 0 (even): down
+    (0x3F818000, 0x3F82),  # exact tie, kept LSB 1 (odd): up
+    (0x3F808001, 0x3F81),  # just above the tie: up
+    (0x3F807FFF, 0x3F80),  # just below the tie: down
+    (0xBF818000, 0xBF82),  # negative tie, odd: magnitude up, sign kept
+    (0xBF808000, 0xBF80),  # negative tie, even: down
+    (0x3FFF8000, 0x4000),  # tie with odd LSB carries into the exponent: 2.0
+    (0x7F7F7FFF, 0x7F7F),  # largest finite bf16 from below
+    (0x7F7F8000, 0x7F80),  # tie at the largest finite, odd: rounds to +inf
+    (0x00008000, 0x0000),  # subnormal tie, even: +0
+    (0x00018000, 0x0002),  # subnormal tie, odd: up
+    (0x0000FFFF, 0x0001),  # rounds up to the smallest bf16 subnormal
+    (0x00010001, 0x0001),  # just above the smallest subnormal: down
+    (0x80000000, 0x8000),  # -0 stays -0
+    (0x80008000, 0x8000),  # negative subnormal tie, even: -0
+]
+
+
+def test_bf16_round_hand_worked_bit_patterns():
+    bits = np.array([b for b, _ in BF16_HAND], np.uint32)
+    want = np.array([w for _, w in BF16_HAND], np.uint32) << 16
+    got = O.bf16_round(bits.view(np.float32)).view(np.uint32)
+    np.testing.assert_array_equal(got, want)
+
+
+def test_bf16_round_equals_exact_round_to_nearest_even():
+    """Random finite float32 values across the whole exponent range, plus values placed exactly on,
+    one ulp below and one ulp above bf16 rounding ties, against the exact-arithmetic rounding."""
+    rng = np.random.default_rng(51)
+    u = rng.integers(0, 2 ** 32, 4000, dtype=np.uint64).astype(np.uint32)
+    u = u[((u >> 23) & 0xFF) != 0xFF]                             # finite only
+    ties = (rng.integers(0, 2 ** 16, 1000, dtype=np.uint64).astype(np.uint32) << 16) | 0x8000
+    ties = ties[((ties >> 23) & 0xFF) != 0xFF]
+    x = np.concatenate([u, ties, ties - 1, ties + 1]).view(np.float32)
+    got = O.bf16_round(x)
+    want = np.array([_bf16_by_definition(v) for v in x], np.float64)
+    np.testing.assert_array_equal(got.astype(np.float64), want)
+    # sign of zero results follows the input's sign
+    zero = got == 0
+    np.testing.assert_array_equal(np.signbit(got[zero]), np.signbit(x[zero]))
+
+
+def test_bf16_round_agrees_with_torch_on_a_wide_sweep():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(52)
+    u = rng.integers(0, 2 ** 32, 300000, dtype=np.uint64).astype(np.uint32)
+    x = u[((u >> 23) & 0xFF) != 0xFF].view(np.float32)
+    t = torch.from_numpy(x.copy()).to(torch.bfloat16).to(torch.float32).numpy()
+    np.testing.assert_array_equal(O.bf16_round(x).view(np.uint32), t.view(np.uint32))
+
+
+def test_bf16_bits_to_f64_decodes_every_pattern():
+    """All 65536 bf16 patterns against sign * (1 + m/128) * 2^(e - 127) (normal), sign * m/128 * 2^-126
+    (subnormal), +-inf and NaN."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    with np.errstate(invalid="ignore"):
+        got = O.bf16_bits_to_f64(bits)
+    for b in range(65536):
+        s, e, m = b >> 15, (b >> 7) & 0xFF, b & 0x7F
+        sign = -1.0 if s else 1.0
+        if e == 0xFF:
+            if m == 0:
+                assert got[b] == sign * float("inf")
+            else:
+                assert np.isnan(got[b])
+            continue
+        mag = Fraction(m, 128) * Fraction(2) ** -126 if e == 0 else (1 + Fraction(m, 128)) * Fraction(2) ** (e - 127)
+        assert got[b] == sign * float(mag), hex(b)
+        if mag == 0:
+            assert bool(np.signbit(got[b])) == bool(s)
+
+
+def _dequant_entry_by_definition(codes_tn, scales, part):
+    """One entry of the training weights: stage terms added in float32 (each partial sum rounded to
+    nearest-even float32) in stage order from 0, then rounded once to bf16.  part 0: real, 1: imag."""
+    acc = Fraction(0)
+    for t, k in enumerate(codes_tn):
+        if (k & 1) != part:
+            continue                              # this stage's code lies on the other axis
+        term = Fraction(float(scales[t][part])) * (-1 if k >> 1 else 1)
+        acc = _rne(acc + term, 24, -126)
+    return float(_rne(acc, 8, -126))
+
+
+@pytest.mark.parametrize("T", [2, 3])
+def test_dequantize_bf16_multi_stage_equals_exact_stage_order_sum(T):
+    rng = np.random.default_rng(60 + T)
+    k = rng.integers(0, 4, (T, 6, 40))
+    packed = O.pack_codes(k)
+    sc = rng.uniform(0.001, 0.05, (T, 2)).astype(np.float32)
+    re, im = O.dequantize_bf16(packed, sc)
+    for n in range(k.shape[1]):
+        for j in range(k.shape[2]):
+            col = [int(k[t, n, j]) for t in range(T)]
+            assert re[n, j] == _dequant_entry_by_definition(col, sc, 0), (n, j)
+            assert im[n, j] == _dequant_entry_by_definition(col, sc, 1), (n, j)
+
+
+def test_dequantize_bf16_rounds_each_stage_sum_in_float32():
+    """Hand-worked: real-axis codes with scales 1 + 2^-8, 2^-25, 2^-25.  In float32 each 2^-25 added
+    to 1 + 2^-8 is a tie that rounds back to the even 1 + 2^-8, whose bf16 rounding is again a tie,
+    to 1.0.  The exact sum 1 + 2^-8 + 2^-24 would round to 1 + 2^-7 instead."""
+    sc = np.array([[1 + 2.0 ** -8, 0.5], [2.0 ** -25, 0.5], [2.0 ** -25, 0.5]], np.float32)
+    packed = O.pack_codes(np.zeros((3, 1, 4), np.uint8))       # code 0 (+1) at every stage
+    re, im = O.dequantize_bf16(packed, sc)
+    np.testing.assert_array_equal(re, np.ones((1, 4), np.float32))
+    np.testing.assert_array_equal(im, np.zeros((1, 4), np.float32))
+    assert float(_rne(Fraction(1) + Fraction(1, 256) + Fraction(1, 2 ** 24), 8, -126)) == 1 + 2.0 ** -7

@@ -24,8 +24,13 @@ def test_static_scratch_limit_is_checked_on_the_host():
     assert lib.ifq_quantize_workspace_bytes(arr, 1, 2) > Q.IFQ_QUANT_STATIC_SCRATCH_BYTES
     assert _static([big], 2) == 10
     assert Q.ifq_status_string(10)
-    # just above the limit: one tensor whose partials alone exceed it
-    edge = L.QTensor(FAKE, FAKE, 4096 * 65536 // 1024 + 1, 1024, FAKE, FAKE)
+    # the limit itself: 262144 x 1024 complex weights need exactly the fixed scratch (32 bytes per
+    # 4096 weights); checked on the sizes alone, since a call with these fake pointers would launch
+    at = L.QTensor(FAKE, FAKE, 262144, 1024, FAKE, FAKE)
+    assert lib.ifq_quantize_workspace_bytes((L.QTensor * 1)(at), 1, 1) == Q.IFQ_QUANT_STATIC_SCRATCH_BYTES
+    # one row more is refused before anything is launched
+    edge = L.QTensor(FAKE, FAKE, 262144 + 1, 1024, FAKE, FAKE)
+    assert lib.ifq_quantize_workspace_bytes((L.QTensor * 1)(edge), 1, 1) > Q.IFQ_QUANT_STATIC_SCRATCH_BYTES
     assert _static([edge], 1) == 10
     # the usual argument errors come first, as for ifq_quantize_pack
     assert _static([L.QTensor(FAKE, None, 64, 128, FAKE, FAKE)], 1) == 1
