@@ -2,7 +2,8 @@
 
 The compute path is the CUDA library libifq.so (include/ifq.h); this package
 holds its ctypes binding (_lib), the in-tree build script (build) and the
-seeded synthetic workload generator (workloads).
+seeded synthetic workload generator (workloads), and the host side of the
+row split of a tensor across GPUs (shard).
 """
 from ._lib import (  # noqa: F401
     EXPORTED,
@@ -12,15 +13,19 @@ from ._lib import (  # noqa: F401
     IFQ_MAX_GROUP,
     IFQ_MAX_STAGES,
     IFQ_QUANT_STATIC_SCRATCH_BYTES,
+    GemvPlan,
     IfqError,
     LayerSet,
     LIB_PATH,
     ifq_dequantize,
     ifq_gemm,
+    ifq_gemm_wait_limit,
     ifq_gemv,
     ifq_gemv_workspace_bytes,
     ifq_quantize_pack,
+    ifq_quantize_finish,
     ifq_quantize_pack_static,
+    ifq_quantize_stage,
     ifq_quantize_workspace_bytes,
     ifq_status_string,
     ifq_widely_linear_from_real,

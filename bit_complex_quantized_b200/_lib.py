@@ -26,12 +26,18 @@ EXPORTED = (
     "ifq_quantize_workspace_bytes",
     "ifq_quantize_pack",
     "ifq_quantize_pack_static",
+    "ifq_quantize_stage",
+    "ifq_quantize_finish",
     "ifq_widely_linear_quantize_workspace_bytes",
     "ifq_widely_linear_quantize_pack",
     "ifq_dequantize",
     "ifq_gemv_workspace_bytes",
     "ifq_gemv",
+    "ifq_gemv_plan_bytes",
+    "ifq_gemv_prepare",
+    "ifq_gemv_run",
     "ifq_gemm",
+    "ifq_gemm_wait_limit",
 )
 
 STATUS_NAMES = {
@@ -50,6 +56,11 @@ class IfqError(RuntimeError):
 class QTensor(ctypes.Structure):
     _fields_ = [("w_re", ctypes.c_void_p), ("w_im", ctypes.c_void_p), ("N", ctypes.c_int64),
                 ("K", ctypes.c_int64), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+class QPartials(ctypes.Structure):
+    _fields_ = [("partials", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("scales", ctypes.c_void_p)]
 
 
 class DqTensor(ctypes.Structure):
@@ -93,6 +104,10 @@ def load():
     lib.ifq_quantize_pack.argtypes = [ctypes.POINTER(QTensor), i32, i32, vp, sz, vp, vp]
     lib.ifq_quantize_pack_static.restype = i32
     lib.ifq_quantize_pack_static.argtypes = [ctypes.POINTER(QTensor), i32, i32, vp, vp]
+    lib.ifq_quantize_stage.restype = i32
+    lib.ifq_quantize_stage.argtypes = [ctypes.POINTER(QTensor), i32, i32, vp, sz, vp, vp]
+    lib.ifq_quantize_finish.restype = i32
+    lib.ifq_quantize_finish.argtypes = [ctypes.POINTER(QPartials), i32, i32, vp]
     lib.ifq_widely_linear_quantize_workspace_bytes.restype = sz
     lib.ifq_widely_linear_quantize_workspace_bytes.argtypes = [ctypes.POINTER(WlLayer), i32, i32]
     lib.ifq_widely_linear_quantize_pack.restype = i32
@@ -103,8 +118,16 @@ def load():
     lib.ifq_gemv_workspace_bytes.argtypes = [ctypes.POINTER(Layer), i32, i32, i32]
     lib.ifq_gemv.restype = i32
     lib.ifq_gemv.argtypes = [ctypes.POINTER(Layer), i32, i32, i32, vp, sz, vp, vp]
+    lib.ifq_gemv_plan_bytes.restype = sz
+    lib.ifq_gemv_plan_bytes.argtypes = []
+    lib.ifq_gemv_prepare.restype = i32
+    lib.ifq_gemv_prepare.argtypes = [ctypes.POINTER(Layer), i32, i32, i32, vp, sz, vp, vp, sz]
+    lib.ifq_gemv_run.restype = i32
+    lib.ifq_gemv_run.argtypes = [vp, vp]
     lib.ifq_gemm.restype = i32
     lib.ifq_gemm.argtypes = [ctypes.POINTER(Layer), i32, i32, i64, vp, vp]
+    lib.ifq_gemm_wait_limit.restype = i32
+    lib.ifq_gemm_wait_limit.argtypes = [ctypes.POINTER(Layer), i32, i32, i64, ctypes.c_uint64, vp, vp]
     _lib = lib
     return lib
 
@@ -161,6 +184,22 @@ def ifq_quantize_pack_static(tensors, T, dev_status=None, stream=None):
     """As ifq_quantize_pack, with the library's fixed device scratch instead of a workspace."""
     arr = _qtensors(tensors)
     _check(load().ifq_quantize_pack_static(arr, len(tensors), T, _ptr(dev_status), _stream(stream)))
+
+
+def ifq_quantize_stage(tensors, t, partials, dev_status=None, stream=None):
+    """Stage t (1-based) of a row shard: codes of the shard and its tile partials in `partials`
+    (a device buffer of ifq_quantize_workspace_bytes(tensors, t) bytes)."""
+    arr = _qtensors(tensors)
+    _check(load().ifq_quantize_stage(arr, len(tensors), t, _ptr(partials),
+                                     partials.numel() * partials.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def ifq_quantize_finish(parts, t, stream=None):
+    """parts: list of (gathered partials of a whole tensor, N, K, scales [T][2]); writes stage t's scales."""
+    arr = (QPartials * len(parts))()
+    for i, (pt, N, K, sc) in enumerate(parts):
+        arr[i] = QPartials(pt.data_ptr(), N, K, sc.data_ptr())
+    _check(load().ifq_quantize_finish(arr, len(parts), t, _stream(stream)))
 
 
 def ifq_dequantize(tensors, T, stream=None):
@@ -243,10 +282,38 @@ def ifq_gemv(layers, T, B, workspace=None, dev_status=None, stream=None, workspa
     _check(load().ifq_gemv(arr, n, T, B, _ptr(workspace), nbytes, _ptr(dev_status), _stream(stream)))
 
 
+class GemvPlan:
+    """A prepared decode call (ifq_gemv_prepare) in a 64-byte aligned host buffer; run() launches it
+    (ifq_gemv_run).  The layers' tensors, the workspace and dev_status must stay alive and in place."""
+
+    def __init__(self, layers, T, B, workspace=None, dev_status=None, workspace_bytes=None):
+        lib = load()
+        n = int(lib.ifq_gemv_plan_bytes())
+        self._buf = ctypes.create_string_buffer(n + 64)
+        addr = ctypes.addressof(self._buf)
+        self.ptr = ctypes.c_void_p((addr + 63) & ~63)
+        self._keep = (layers, workspace, dev_status)
+        nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        if workspace_bytes is not None:
+            nbytes = workspace_bytes
+        arr, cnt = _as_array(layers)
+        self._arr = arr
+        _check(lib.ifq_gemv_prepare(arr, cnt, T, B, _ptr(workspace), nbytes, _ptr(dev_status), self.ptr, n))
+
+    def run(self, stream=None):
+        _check(load().ifq_gemv_run(self.ptr, _stream(stream)))
+
+
 def ifq_gemm(layers, T, M, dev_status=None, stream=None):
     """As ifq_gemv with x [M][K] and y [M][N]."""
     arr, n = _as_array(layers)
     _check(load().ifq_gemm(arr, n, T, M, _ptr(dev_status), _stream(stream)))
+
+
+def ifq_gemm_wait_limit(layers, T, M, wait_limit_ns, dev_status=None, stream=None):
+    """As ifq_gemm with each pipeline wait bounded by wait_limit_ns (IFQ_DEV_TIMEOUT when one runs out)."""
+    arr, n = _as_array(layers)
+    _check(load().ifq_gemm_wait_limit(arr, n, T, M, int(wait_limit_ns), _ptr(dev_status), _stream(stream)))
 
 
 # Raw entry point for callers that build ctypes descriptors themselves.

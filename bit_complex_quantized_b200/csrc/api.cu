@@ -1,8 +1,10 @@
 // C ABI of libifq: argument validation, then one enqueue per entry point.
 // Every error is returned before anything is launched.
 #include <cuda_runtime.h>
+#include <string.h>
 
 #include "../../include/ifq.h"
+#include "ifq_common.cuh"
 #include "ifq_internal.h"
 
 namespace {
@@ -33,11 +35,23 @@ ifq_status check_layers(const ifq_layer* L, int count, int T) {
     if (!l.codes_u || !l.scales_u || !l.x_re || !l.x_im || !l.y_re || !l.y_im) return IFQ_ERR_NULL;
     if ((l.codes_w == nullptr) != (l.scales_w == nullptr)) return IFQ_ERR_NULL;
     if ((l.rot_re == nullptr) != (l.rot_im == nullptr)) return IFQ_ERR_NULL;
-    if (l.N < 1 || l.K < 64 || (l.K % 64) != 0) return IFQ_ERR_SHAPE;
+    if (l.N < 1 || l.K < 4 || (l.K % 4) != 0) return IFQ_ERR_SHAPE;
     if (l.N > (int64_t)1 << 30 || l.K > (int64_t)1 << 30) return IFQ_ERR_SHAPE;
     if (!aligned16(l.codes_u) || (l.codes_w && !aligned16(l.codes_w)) || !aligned16(l.x_re) || !aligned16(l.x_im) ||
         !aligned16(l.y_re) || !aligned16(l.y_im) || (reinterpret_cast<uintptr_t>(l.scales_u) & 3u) ||
         (reinterpret_cast<uintptr_t>(l.scales_w) & 3u) || (l.rot_re && (!aligned16(l.rot_re) || !aligned16(l.rot_im))))
+      return IFQ_ERR_ALIGN;
+  }
+  return IFQ_OK;
+}
+
+ifq_status check_qtensors(const ifq_qtensor* tensors, int count) {
+  for (int i = 0; i < count; ++i) {
+    const ifq_qtensor& t = tensors[i];
+    if (!t.w_re || !t.w_im || !t.codes || !t.scales) return IFQ_ERR_NULL;
+    if (t.N < 1 || t.K < 4 || (t.K % 4) != 0) return IFQ_ERR_SHAPE;
+    if (t.K > (int64_t)1 << 30 || t.N > ((int64_t)1 << 40) / t.K) return IFQ_ERR_SHAPE;
+    if (!aligned16(t.w_re) || !aligned16(t.w_im) || !aligned16(t.codes) || (reinterpret_cast<uintptr_t>(t.scales) & 3u))
       return IFQ_ERR_ALIGN;
   }
   return IFQ_OK;
@@ -88,19 +102,43 @@ ifq_status ifq_quantize_pack(const ifq_qtensor* tensors, int count, int T, void*
   if (!tensors) return IFQ_ERR_NULL;
   if (count < 1 || count > IFQ_MAX_GROUP) return IFQ_ERR_COUNT;
   if (T < 1 || T > IFQ_MAX_STAGES) return IFQ_ERR_STAGES;
-  for (int i = 0; i < count; ++i) {
-    const ifq_qtensor& t = tensors[i];
-    if (!t.w_re || !t.w_im || !t.codes || !t.scales) return IFQ_ERR_NULL;
-    if (t.N < 1 || t.K < 4 || (t.K % 4) != 0) return IFQ_ERR_SHAPE;
-    if (t.K > (int64_t)1 << 30 || t.N > ((int64_t)1 << 40) / t.K) return IFQ_ERR_SHAPE;
-    if (!aligned16(t.w_re) || !aligned16(t.w_im) || !aligned16(t.codes) || (reinterpret_cast<uintptr_t>(t.scales) & 3u))
-      return IFQ_ERR_ALIGN;
-  }
+  ifq_status st0 = check_qtensors(tensors, count);
+  if (st0 != IFQ_OK) return st0;
   if (!workspace || workspace_bytes < ifq::quant_workspace_bytes(tensors, count)) return IFQ_ERR_WORKSPACE;
   if (!aligned16(workspace)) return IFQ_ERR_ALIGN;
   ifq_status st = check_device();
   if (st != IFQ_OK) return st;
   return from_cuda(ifq::launch_quantize(tensors, count, T, workspace, dev_status, as_stream(stream)));
+}
+
+ifq_status ifq_quantize_stage(const ifq_qtensor* tensors, int count, int t, void* partials, size_t partials_bytes,
+                              uint32_t* dev_status, ifq_stream_t stream) {
+  if (!tensors) return IFQ_ERR_NULL;
+  if (count < 1 || count > IFQ_MAX_GROUP) return IFQ_ERR_COUNT;
+  if (t < 1 || t > IFQ_MAX_STAGES) return IFQ_ERR_STAGES;
+  ifq_status st = check_qtensors(tensors, count);
+  if (st != IFQ_OK) return st;
+  if (!partials || partials_bytes < ifq::quant_workspace_bytes(tensors, count)) return IFQ_ERR_WORKSPACE;
+  if (!aligned16(partials)) return IFQ_ERR_ALIGN;
+  st = check_device();
+  if (st != IFQ_OK) return st;
+  return from_cuda(ifq::launch_quantize_stage(tensors, count, t - 1, partials, dev_status, as_stream(stream)));
+}
+
+ifq_status ifq_quantize_finish(const ifq_qpartials* parts, int count, int t, ifq_stream_t stream) {
+  if (!parts) return IFQ_ERR_NULL;
+  if (count < 1 || count > IFQ_MAX_GROUP) return IFQ_ERR_COUNT;
+  if (t < 1 || t > IFQ_MAX_STAGES) return IFQ_ERR_STAGES;
+  for (int i = 0; i < count; ++i) {
+    const ifq_qpartials& q = parts[i];
+    if (!q.partials || !q.scales) return IFQ_ERR_NULL;
+    if (q.N < 1 || q.K < 4 || (q.K % 4) != 0) return IFQ_ERR_SHAPE;
+    if (q.K > (int64_t)1 << 30 || q.N > ((int64_t)1 << 40) / q.K) return IFQ_ERR_SHAPE;
+    if (!aligned16(q.partials) || (reinterpret_cast<uintptr_t>(q.scales) & 3u)) return IFQ_ERR_ALIGN;
+  }
+  ifq_status st = check_device();
+  if (st != IFQ_OK) return st;
+  return from_cuda(ifq::launch_quantize_finish(parts, count, t - 1, as_stream(stream)));
 }
 
 ifq_status ifq_quantize_pack_static(const ifq_qtensor* tensors, int count, int T, uint32_t* dev_status,
@@ -181,8 +219,9 @@ ifq_status ifq_dequantize(const ifq_dqtensor* tensors, int count, int T, ifq_str
 
 size_t ifq_gemv_workspace_bytes(const ifq_layer* layers, int count, int T, int B) {
   if (check_layers(layers, count, T) != IFQ_OK || B < 1 || B > IFQ_MAX_GEMV_BATCH) return 0;
-  return B <= ifq::IFQ_I8_MAX_BATCH ? ifq::gemv_i8_workspace_bytes(layers, count, T, B)
-                                    : ifq::gemv_bf16_workspace_bytes(layers, count, B);
+  if (ifq::any_narrow_k(layers, count)) return 0;
+  return B <= ifq::IFQ_FP4_MAX_BATCH ? ifq::gemv_fp4_workspace_bytes(layers, count, T, B)
+                                     : ifq::gemv_bf16_workspace_bytes(layers, count, B);
 }
 
 ifq_status ifq_gemv(const ifq_layer* layers, int count, int T, int B, void* workspace, size_t workspace_bytes,
@@ -190,28 +229,106 @@ ifq_status ifq_gemv(const ifq_layer* layers, int count, int T, int B, void* work
   ifq_status st = check_layers(layers, count, T);
   if (st != IFQ_OK) return st;
   if (B < 1 || B > IFQ_MAX_GEMV_BATCH) return IFQ_ERR_BATCH;
-  const bool integer = B <= ifq::IFQ_I8_MAX_BATCH;
-  const size_t need = integer ? ifq::gemv_i8_workspace_bytes(layers, count, T, B)
-                              : ifq::gemv_bf16_workspace_bytes(layers, count, B);
+  if (ifq::any_narrow_k(layers, count)) {
+    st = check_device();
+    if (st != IFQ_OK) return st;
+    return from_cuda(ifq::launch_product_generic(layers, count, T, B, dev_status, as_stream(stream)));
+  }
+  const bool fp4 = B <= ifq::IFQ_FP4_MAX_BATCH;
+  const size_t need = fp4 ? ifq::gemv_fp4_workspace_bytes(layers, count, T, B)
+                          : ifq::gemv_bf16_workspace_bytes(layers, count, B);
   if (need > 0 && (!workspace || workspace_bytes < need)) return IFQ_ERR_WORKSPACE;
   if (need > 0 && !aligned16(workspace)) return IFQ_ERR_ALIGN;
   st = check_device();
   if (st != IFQ_OK) return st;
-  if (integer)
-    return from_cuda(ifq::launch_gemv_i8(layers, count, T, B, workspace, dev_status, as_stream(stream)));
+  if (fp4) return from_cuda(ifq::launch_gemv_fp4(layers, count, T, B, workspace, dev_status, as_stream(stream)));
   return from_cuda(ifq::launch_gemv(layers, count, T, B, workspace, dev_status, as_stream(stream)));
 }
 
-ifq_status ifq_gemm(const ifq_layer* layers, int count, int T, int64_t M, uint32_t* dev_status,
-                    ifq_stream_t stream) {
+// A prepared decode call, in the caller's host buffer: the routing and the descriptors, then (4-bit
+// path) the finished launch parameters at a 64-byte boundary.
+namespace {
+constexpr uint32_t kPlanMagic = 0x50514649u;
+struct alignas(64) GemvPlanHeader {
+  uint32_t magic;
+  int32_t path;  // 0: 4-bit tensor cores, 1: bf16 mma.sync, 2: CUDA cores (narrow K)
+  int32_t count, T, B;
+  void* workspace;
+  uint32_t* dev_status;
+  ifq_layer layers[IFQ_MAX_GROUP];
+};
+constexpr size_t kPlanFp4Offset = (sizeof(GemvPlanHeader) + 63) & ~(size_t)63;
+}  // namespace
+
+size_t ifq_gemv_plan_bytes(void) { return kPlanFp4Offset + ifq::gemv_fp4_plan_bytes(); }
+
+ifq_status ifq_gemv_prepare(const ifq_layer* layers, int count, int T, int B, void* workspace,
+                            size_t workspace_bytes, uint32_t* dev_status, void* plan, size_t plan_bytes) {
+  ifq_status st = check_layers(layers, count, T);
+  if (st != IFQ_OK) return st;
+  if (B < 1 || B > IFQ_MAX_GEMV_BATCH) return IFQ_ERR_BATCH;
+  if (!plan) return IFQ_ERR_NULL;
+  if (plan_bytes < ifq_gemv_plan_bytes()) return IFQ_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(plan) & 63u) return IFQ_ERR_ALIGN;
+  const bool narrow = ifq::any_narrow_k(layers, count);
+  const bool fp4 = !narrow && B <= ifq::IFQ_FP4_MAX_BATCH;
+  const size_t need = narrow ? 0
+                      : fp4  ? ifq::gemv_fp4_workspace_bytes(layers, count, T, B)
+                             : ifq::gemv_bf16_workspace_bytes(layers, count, B);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return IFQ_ERR_WORKSPACE;
+  if (need > 0 && !aligned16(workspace)) return IFQ_ERR_ALIGN;
+  st = check_device();
+  if (st != IFQ_OK) return st;
+  GemvPlanHeader* h = static_cast<GemvPlanHeader*>(plan);
+  memset(h, 0, sizeof(GemvPlanHeader));
+  h->path = narrow ? 2 : fp4 ? 0 : 1;
+  h->count = count;
+  h->T = T;
+  h->B = B;
+  h->workspace = workspace;
+  h->dev_status = dev_status;
+  memcpy(h->layers, layers, sizeof(ifq_layer) * count);
+  if (fp4) {
+    const cudaError_t e = ifq::plan_gemv_fp4(layers, count, T, B, workspace, dev_status,
+                                             static_cast<char*>(plan) + kPlanFp4Offset);
+    if (e != cudaSuccess) return IFQ_ERR_CUDA;
+  }
+  h->magic = kPlanMagic;
+  return IFQ_OK;
+}
+
+ifq_status ifq_gemv_run(const void* plan, ifq_stream_t stream) {
+  if (!plan) return IFQ_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(plan) & 63u) return IFQ_ERR_ALIGN;
+  const GemvPlanHeader* h = static_cast<const GemvPlanHeader*>(plan);
+  if (h->magic != kPlanMagic) return IFQ_ERR_NULL;
+  switch (h->path) {
+    case 0: return from_cuda(ifq::run_gemv_fp4_plan(static_cast<const char*>(plan) + kPlanFp4Offset, as_stream(stream)));
+    case 1:
+      return from_cuda(ifq::launch_gemv(h->layers, h->count, h->T, h->B, h->workspace, h->dev_status, as_stream(stream)));
+    default:
+      return from_cuda(ifq::launch_product_generic(h->layers, h->count, h->T, h->B, h->dev_status, as_stream(stream)));
+  }
+}
+
+ifq_status ifq_gemm_wait_limit(const ifq_layer* layers, int count, int T, int64_t M, uint64_t wait_limit_ns,
+                               uint32_t* dev_status, ifq_stream_t stream) {
   ifq_status st = check_layers(layers, count, T);
   if (st != IFQ_OK) return st;
   if (M < 1 || M > ((int64_t)1 << 31) - 128) return IFQ_ERR_BATCH;
   for (int i = 0; i < count; ++i)
     if ((int64_t)T * layers[i].N > ((int64_t)1 << 31) - 64) return IFQ_ERR_SHAPE;
+  if (wait_limit_ns == 0) return IFQ_ERR_SHAPE;
   st = check_device();
   if (st != IFQ_OK) return st;
-  return from_cuda(ifq::launch_gemm(layers, count, T, M, dev_status, as_stream(stream)));
+  if (ifq::any_narrow_k(layers, count))
+    return from_cuda(ifq::launch_product_generic(layers, count, T, M, dev_status, as_stream(stream)));
+  return from_cuda(ifq::launch_gemm(layers, count, T, M, wait_limit_ns, dev_status, as_stream(stream)));
+}
+
+ifq_status ifq_gemm(const ifq_layer* layers, int count, int T, int64_t M, uint32_t* dev_status,
+                    ifq_stream_t stream) {
+  return ifq_gemm_wait_limit(layers, count, T, M, IFQ_WAIT_LIMIT_NS, dev_status, stream);
 }
 
 }  // extern "C"

@@ -70,6 +70,7 @@ struct __align__(64) GemmArgs {
   const float* rot[2];  // optional epilogue rotation [M][N] (re, im), or null
   int64_t N, K, M;
   int T, nbranch;
+  uint64_t wait_ns;  // limit of each pipeline wait (drains after a lost wait keep IFQ_WAIT_LIMIT_NS)
   uint32_t* status;
 };
 
@@ -147,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         for (int kb = 0; kb < KB; ++kb) {
           const int it = p * KB + kb, s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!mbar_wait_bounded(&S->empty[s], ph ^ 1u, abort)) break;
+          if (!mbar_wait_bounded_ns(&S->empty[s], ph ^ 1u, abort, a.wait_ns)) break;
           mbar_arrive_expect_tx(&S->full_tma[s], kTmaBytes);
           tma_load_2d(xtile(s), &a.tmap_x[0], kb * BK, (int32_t)m0, &S->full_tma[s]);
           tma_load_2d(xtile(s) + kTileX, &a.tmap_x[1], kb * BK, (int32_t)m0, &S->full_tma[s]);
@@ -163,36 +164,37 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       }
     }
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      for (int p = 0; p < P && !*abort; ++p) {
-        // the epilogue has read the previous (stage, branch) accumulator
-        if (!mbar_wait_bounded(&S->acc_empty, ((uint32_t)p & 1u) ^ 1u, abort)) break;
-        tc_fence_after();
-        bool ok = true;
-        for (int kb = 0; kb < KB; ++kb) {
-          const int it = p * KB + kb, s = it % STAGES;
-          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!mbar_wait_bounded(&S->full_tma[s], ph, abort) || !mbar_wait_bounded(&S->full_a[s], ph, abort)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t xb = smem_u32(xtile(s));
-#pragma unroll
-          for (int ks = 0; ks < BK / 16; ++ks)
-            umma_bf16_ta(tmem, tmem + kAcol + 32 * s + 8 * ks, umma_desc_sw128(xb + ks * 32), kIdesc,
-                         (kb | ks) != 0);
-          umma_commit(&S->empty[s]);
-        }
+    // ------------------------------------------------------------ MMA issuer (whole warp, one elected lane issues)
+    const uint64_t xdesc0 = umma_desc_sw128(smem_u32(xtile(0)));
+    for (int p = 0; p < P; ++p) {
+      // the epilogue has read the previous (stage, branch) accumulator
+      int ok = 1;
+      if (lane == 0) ok = !*abort && mbar_wait_bounded_ns(&S->acc_empty, ((uint32_t)p & 1u) ^ 1u, abort, a.wait_ns);
+      ok = __shfl_sync(0xffffffffu, ok, 0);  // every lane takes lane 0's result: the warp stays converged
+      if (!ok) break;
+      tc_fence_after();
+      for (int kb = 0; kb < KB; ++kb) {
+        const int it = p * KB + kb, s = it % STAGES;
+        const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+        if (lane == 0)
+          ok = mbar_wait_bounded_ns(&S->full_tma[s], ph, abort, a.wait_ns) &&
+               mbar_wait_bounded_ns(&S->full_a[s], ph, abort, a.wait_ns);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        umma_commit(&S->acc_full);
+        tc_fence_after();
+        // the four K16 steps of the stage: B advances 32 bytes (2 descriptor units) per step inside the
+        // 128-byte swizzle row, A 8 TMEM columns
+        umma_bf16_ta_x4(tmem, tmem + kAcol + 32 * s, xdesc0 + (uint64_t)((uint32_t)s * (kStageBytes >> 4)), kIdesc,
+                        kb != 0);
+        umma_commit_elect(&S->empty[s]);
       }
-      if (*abort) {
-        volatile int never = 0;
-        umma_commit(&S->drain);
-        mbar_wait_bounded(&S->drain, 0u, &never);
-      }
+      if (!ok) break;
+      umma_commit_elect(&S->acc_full);
+    }
+    if (lane == 0 && *abort) {
+      volatile int never = 0;
+      umma_commit(&S->drain);
+      mbar_wait_bounded(&S->drain, 0u, &never);
     }
   } else if (warp < kExpWarps) {
     // ------------------------------------------------------------ expanders
@@ -205,7 +207,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
         int ok = 1;
         if (lane == 0)
-          ok = mbar_wait_bounded(&S->empty[s], ph ^ 1u, abort) && mbar_wait_bounded(&S->full_tma[s], ph, abort);
+          ok = mbar_wait_bounded_ns(&S->empty[s], ph ^ 1u, abort, a.wait_ns) &&
+               mbar_wait_bounded_ns(&S->full_tma[s], ph, abort, a.wait_ns);
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         // Rows past N carry other stages' or no codes; their outputs are never stored.
         const uint4 cw = *reinterpret_cast<const uint4*>(ctile(s) + o * 16);
@@ -229,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
     for (int p = 0; p < P && !__shfl_sync(0xffffffffu, *abort, 0); ++p) {
       int ok = 1;
-      if (lane == 0) ok = mbar_wait_bounded(&S->acc_full, (uint32_t)p & 1u, abort);
+      if (lane == 0) ok = mbar_wait_bounded_ns(&S->acc_full, (uint32_t)p & 1u, abort, a.wait_ns);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       tc_fence_after();
       const int t = p / a.nbranch, br = p % a.nbranch;
@@ -377,7 +380,8 @@ bool encode_tiled_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const vo
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-cudaError_t launch_gemm(const ifq_layer* Ls, int count, int T, int64_t M, uint32_t* dev_status, cudaStream_t s) {
+cudaError_t launch_gemm(const ifq_layer* Ls, int count, int T, int64_t M, uint64_t wait_ns, uint32_t* dev_status,
+                        cudaStream_t s) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
@@ -394,6 +398,7 @@ cudaError_t launch_gemm(const ifq_layer* Ls, int count, int T, int64_t M, uint32
     a.M = M;
     a.T = T;
     a.status = dev_status;
+    a.wait_ns = wait_ns;
     a.scales[0] = L.scales_u;
     a.scales[1] = L.scales_w;
     a.y[0] = L.y_re;

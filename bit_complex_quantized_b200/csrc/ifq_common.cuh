@@ -95,6 +95,20 @@ IFQ_DEVINL bool mbar_wait_bounded_sleep(uint64_t* bar, uint32_t parity, volatile
   }
 }
 
+// As mbar_wait_bounded, with a caller-chosen limit in nanoseconds instead of IFQ_WAIT_LIMIT_NS.
+IFQ_DEVINL bool mbar_wait_bounded_ns(uint64_t* bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_ns() - t0 > limit_ns) {
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
 // Waits until the phase with the given parity has completed.  Gives up and
 // returns false after IFQ_WAIT_LIMIT_NS, or as soon as *abort is seen set by
 // another thread of the CTA; on a timeout it sets *abort itself.
@@ -173,6 +187,33 @@ IFQ_DEVINL void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, 
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Four kind::f16 MMAs with A in TMEM (columns a_tmem + 8 c) and B in shared memory (descriptor b_desc
+// + 2 c: 32 bytes further inside a 128-byte swizzle row), c = 0..3, from one elected lane of a
+// converged warp; the first accumulates only if `accumulate`, the others always.
+IFQ_DEVINL void umma_bf16_ta_x4(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, %4, %4;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %6, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %8, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%9], %10, %3, t;\n\t"
+      "}" ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(a_tmem + 8u), "l"(b_desc + 2u),
+      "r"(a_tmem + 16u), "l"(b_desc + 4u), "r"(a_tmem + 24u), "l"(b_desc + 6u)
+      : "memory");
+}
+
+// tcgen05.commit from one elected lane of a converged warp.
+IFQ_DEVINL void umma_commit_elect(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
       : "memory");
 }
 

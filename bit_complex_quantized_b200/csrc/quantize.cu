@@ -475,6 +475,45 @@ cudaError_t launch_quantize(const ifq_qtensor* t, int count, int T, void* ws, ui
   return launch_stages(p, 0, T, false, s);
 }
 
+// One stage of the quantizer on row shards of the tensors (a tensor's rows split across GPUs): the
+// stage kernel writes the shard's codes of `stage` and one partial per tile of the shard into
+// `partials`, without the reduction.
+cudaError_t launch_quantize_stage(const ifq_qtensor* t, int count, int stage, void* partials, uint32_t* dev_status,
+                                  cudaStream_t s) {
+  QParams p;
+  const int64_t tiles = fill_qparams(t, count, partials, p);
+  p.status = dev_status;
+  p.stage = stage;
+  if (tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  switch (stage) {
+    case 0: return launch_stage<0>(p, false, s);
+    case 1: return launch_stage<1>(p, false, s);
+    case 2: return launch_stage<2>(p, false, s);
+    case 3: return launch_stage<3>(p, false, s);
+    case 4: return launch_stage<4>(p, false, s);
+    case 5: return launch_stage<5>(p, false, s);
+    case 6: return launch_stage<6>(p, false, s);
+    default: return launch_stage<7>(p, false, s);
+  }
+}
+
+// The stage's scales of whole tensors from the tile partials of all their shards, gathered in row order:
+// the same reduction kernel, over the same tiles in the same order, as ifq_quantize_pack.
+cudaError_t launch_quantize_finish(const ifq_qpartials* q, int count, int stage, cudaStream_t s) {
+  QParams p;
+  memset(&p, 0, sizeof(p));
+  p.count = count;
+  p.stage = stage;
+  for (int i = 0; i < count; ++i) {
+    QTensorArg& a = p.t[i];
+    a.partials = reinterpret_cast<QPartial*>(const_cast<void*>(q[i].partials));
+    a.scales = q[i].scales;
+    a.nquads = q[i].N * q[i].K / 4;
+    a.nblocks = quant_blocks_for(q[i].N, q[i].K);
+  }
+  return launch(quant_reduce_kernel, (unsigned)count, 0, false, p, s);
+}
+
 size_t widely_linear_quant_workspace_bytes(const ifq_wl_layer* Ls, int count) {
   ifq_qtensor t[IFQ_MAX_GROUP];
   fused_tensors(Ls, count, t);

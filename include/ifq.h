@@ -130,6 +130,51 @@ ifq_status ifq_quantize_pack(const ifq_qtensor* tensors, int count, int T, void*
                              size_t workspace_bytes, uint32_t* dev_status, ifq_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * ifq_quantize_stage, ifq_quantize_finish  ("Fairy2i write-up" §3.2, §4.1; rows
+ * of a tensor split across GPUs)
+ *
+ * ifq_quantize_pack in two halves per stage, for a tensor whose rows are split
+ * across GPUs.  A stage's scales are means over the whole tensor (§3.2), so the
+ * shards exchange the stage's tile partials before the next stage:
+ *   1. every GPU: ifq_quantize_stage(shard, t) -- stage t's codes of its rows and
+ *      one 32-byte partial (class sums and count) per 4096-weight tile of the
+ *      shard, in `partials`;
+ *   2. gather the partials of all shards in row order (e.g. an all-gather);
+ *   3. every GPU: ifq_quantize_finish(gathered partials of the whole tensor, t)
+ *      -- stage t's scales, by the same reduction over the same tiles in the
+ *      same order as ifq_quantize_pack.
+ * When every shard but the last holds a multiple of 4096 weights (rows * K),
+ * the shards' tiles are exactly the whole tensor's tiles and codes and scales
+ * equal those of ifq_quantize_pack on the whole tensor bit for bit.
+ *
+ *   tensors[i]      the shard: w_re, w_im [N_shard][K]; codes [T][N_shard][K/4]
+ *                   (stage t written, stages < t read); scales [T][2] (stages
+ *                   < t read: the whole tensor's scales, from earlier finish
+ *                   calls).  Sizes and alignment as for ifq_quantize_pack.
+ *   t               the stage, 1..IFQ_MAX_STAGES (stage 1 reads no codes)
+ *   partials        device buffer of ifq_quantize_workspace_bytes(tensors,
+ *                   count, t) bytes (the shard's tile partials, tensor after
+ *                   tensor), 16-byte aligned; no initial contents needed
+ *   parts[i]        .partials: the gathered partials of a whole tensor
+ *                   (quantizer tiles of N x K weights, 32 bytes each, in row
+ *                   order); .N: the whole tensor's rows; .K; .scales: [T][2],
+ *                   stage t written (4-byte aligned)
+ * Errors as for ifq_quantize_pack; t outside 1..IFQ_MAX_STAGES is
+ * IFQ_ERR_STAGES.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  const void* partials;
+  int64_t N;
+  int64_t K;
+  float* scales;
+} ifq_qpartials;
+
+ifq_status ifq_quantize_stage(const ifq_qtensor* tensors, int count, int t, void* partials, size_t partials_bytes,
+                              uint32_t* dev_status, ifq_stream_t stream);
+
+ifq_status ifq_quantize_finish(const ifq_qpartials* parts, int count, int t, ifq_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * ifq_quantize_pack_static
  *
  * The write-ups have no counterpart of this call: it is ifq_quantize_pack
@@ -251,7 +296,10 @@ ifq_status ifq_dequantize(const ifq_dqtensor* tensors, int count, int T, ifq_str
  *
  *   codes_u, scales_u   stage codes and scales of U (required)
  *   codes_w, scales_w   of W, applied to conj(x); both NULL = no conjugate branch
- *   N, K                outputs, inputs: N >= 1, K >= 64, K % 64 == 0
+ *   N, K                outputs, inputs: N >= 1, K >= 4, K % 4 == 0 (the tensor-core
+ *                       kernels take K % 64 == 0; a call with another K runs a
+ *                       plain CUDA-core kernel with float64 sums, and ifq_gemv
+ *                       then needs no workspace)
  *   x_re, x_im          [rows][K] bf16 bit patterns, device, 16-byte aligned
  *   y_re, y_im          [rows][N] float32, device, overwritten
  *   rot_re, rot_im      optional epilogue rotation, both NULL = none: when set,
@@ -314,6 +362,23 @@ size_t ifq_gemv_workspace_bytes(const ifq_layer* layers, int count, int T, int B
 ifq_status ifq_gemv(const ifq_layer* layers, int count, int T, int B, void* workspace, size_t workspace_bytes,
                     uint32_t* dev_status, ifq_stream_t stream);
 
+/* Prepared decode calls, for a caller that repeats the same call (a decode loop): ifq_gemv_prepare
+ * validates the arguments and stores everything the launches need -- the routing, and for the 4-bit
+ * tensor-core path the finished kernel parameters with their tensor maps -- in a caller-owned HOST
+ * buffer of ifq_gemv_plan_bytes() bytes, 64-byte aligned; ifq_gemv_run(plan, stream) then only
+ * launches, and gives the same outputs as ifq_gemv with the same arguments.  Every tensor named by
+ * the layers, the workspace and dev_status must stay allocated and in place while the plan is used
+ * (new activations are written into the same x buffers).  The library keeps nothing: the plan is
+ * the caller's, may be copied bytewise, and runs on any stream of the device it was made on.
+ * Errors: ifq_gemv's; plan NULL is IFQ_ERR_NULL, too small IFQ_ERR_WORKSPACE, misaligned
+ * IFQ_ERR_ALIGN; ifq_gemv_run of a buffer that ifq_gemv_prepare did not fill is IFQ_ERR_NULL. */
+size_t ifq_gemv_plan_bytes(void);
+
+ifq_status ifq_gemv_prepare(const ifq_layer* layers, int count, int T, int B, void* workspace,
+                            size_t workspace_bytes, uint32_t* dev_status, void* plan, size_t plan_bytes);
+
+ifq_status ifq_gemv_run(const void* plan, ifq_stream_t stream);
+
 /* Prefill product for M >= 1 tokens (meant for M >= 128) on the tensor cores:
  * codes are expanded straight into TMEM as exact {-2, 0, +2} bf16 operands (the
  * MMA's A operand), the +-1 and +-i classes accumulate in separate rows of a
@@ -322,6 +387,17 @@ ifq_status ifq_gemv(const ifq_layer* layers, int count, int T, int B, void* work
  * another on the stream.  dev_status may be NULL (timeouts then go unreported). */
 ifq_status ifq_gemm(const ifq_layer* layers, int count, int T, int64_t M, uint32_t* dev_status,
                     ifq_stream_t stream);
+
+/* As ifq_gemm, with every pipeline wait of the tensor-core kernel bounded by
+ * wait_limit_ns (> 0) instead of 2 s.  A wait that runs out sets IFQ_DEV_TIMEOUT
+ * in *dev_status; the kernel then lets its copies and MMAs in flight finish
+ * (waits of up to 2 s), frees its TMEM and returns, so the context stays usable
+ * and the next call runs normally.  The outputs of a call that timed out are
+ * invalid.  For failure-detection tests and for callers with a tighter watchdog
+ * than 2 s; ifq_gemm is this call with 2 s.  wait_limit_ns == 0 is
+ * IFQ_ERR_SHAPE. */
+ifq_status ifq_gemm_wait_limit(const ifq_layer* layers, int count, int T, int64_t M, uint64_t wait_limit_ns,
+                               uint32_t* dev_status, ifq_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -59,12 +59,22 @@ def _call_gemm(layers, T=1, M=128):
 @pytest.mark.parametrize("kw,status", [
     (dict(codes_u=None), 1), (dict(x_re=None), 1), (dict(y_im=None), 1),
     (dict(codes_w=FAKE), 1),                       # W codes without W scales
-    (dict(K=100), 2), (dict(K=0), 2), (dict(N=0), 2), (dict(K=32), 2),
+    (dict(K=102), 2), (dict(K=0), 2), (dict(N=0), 2), (dict(K=2), 2),
     (dict(codes_u=FAKE + 4), 3), (dict(x_im=FAKE + 2), 3), (dict(scales_u=FAKE + 1), 3),
 ])
 def test_gemv_gemm_argument_errors(kw, status):
     assert _call_gemv([_layer(**kw)]) == status
     assert _call_gemm([_layer(**kw)]) == status
+
+
+def test_products_accept_every_width_the_quantizer_accepts():
+    """K % 4 == 0 is enough for the products (narrow widths run the CUDA-core kernel): the shape
+    checks pass and the call stops only at the batch check, before anything is launched."""
+    lib = Q.load()
+    for K in (4, 60, 100, 196, 2052):
+        assert _call_gemv([_layer(K=K)], B=0) == 5
+        assert _call_gemm([_layer(K=K)], M=0) == 5
+        assert lib.ifq_gemv_workspace_bytes((L.Layer * 1)(_layer(K=K)), 1, 2, 1) == 0
 
 
 def test_batch_stage_and_count_errors():
@@ -86,10 +96,12 @@ def test_gemv_workspace_errors():
     arr = (L.Layer * 1)(good)
     need = lib.ifq_gemv_workspace_bytes(arr, 1, 2, 1)
     assert need > 0
-    assert lib.ifq_gemv_workspace_bytes(arr, 1, 2, 2) > need   # integer path up to B = 2, per token
+    # 4-bit tensor-core path up to B = 4: digit tiles, factors and slots grow with the token slots
+    assert lib.ifq_gemv_workspace_bytes(arr, 1, 2, 2) > need
+    assert lib.ifq_gemv_workspace_bytes(arr, 1, 2, 3) == lib.ifq_gemv_workspace_bytes(arr, 1, 2, 4)
     assert _call_gemv([good], T=2, B=2, ws=FAKE, ws_bytes=lib.ifq_gemv_workspace_bytes(arr, 1, 2, 2) - 1) == 6
-    # B >= 3 (bf16 path): partial sums of the K segments of a layer longer than 2048 positions
-    for B in (3, 5, 16):
+    # B >= 5 (bf16 path): partial sums of the K segments of a layer longer than 2048 positions
+    for B in (5, 16):
         assert lib.ifq_gemv_workspace_bytes(arr, 1, 2, B) == (((5504 + 2047) // 2048) * B * 300 * 8 + 255) // 256 * 256
     short = (L.Layer * 1)(_layer(N=300, K=2048))
     assert lib.ifq_gemv_workspace_bytes(short, 1, 2, 5) == 0

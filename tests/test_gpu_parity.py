@@ -448,3 +448,31 @@ def test_prepared_layer_set_gives_the_same_product():
         Q.ifq_gemv(Q.LayerSet([d2]), T, B, workspace=torch.zeros(wsz, dtype=torch.uint8, device=DEV))
         torch.cuda.synchronize()
         assert torch.equal(d1["y_re"], d2["y_re"]) and torch.equal(d1["y_im"], d2["y_im"])
+
+
+@pytest.mark.parametrize("K", [4, 60, 100, 196, 2052])
+def test_products_of_every_width_the_quantizer_accepts(K):
+    """Widths that are multiples of 4 but not of 64 (the CUDA-core kernel), decode and prefill."""
+    rng = np.random.default_rng(K)
+    N, T = 70, 2
+    ws = [_rand_complex(rng, N, K), _rand_complex(rng, N, K, 0.03)]
+    outs = gpu_quantize([(to_dev(a), to_dev(b)) for a, b in ws], T)
+    torch.cuda.synchronize()
+    host = [(c.cpu().numpy(), s.cpu().numpy()) for c, s in outs]
+    for (wr, wi), (cn, sn) in zip(ws, host):
+        check_quantized(wr, wi, cn, sn, T)
+    (cu, su), (cw, sw) = outs
+    (cun, sun), (cwn, swn) = host
+    for rows, gemm in ((1, False), (2, False), (5, False), (16, False), (1, True), (131, True)):
+        xr = torch.from_numpy(rng.standard_normal((rows, K)).astype(np.float32)).to(torch.bfloat16)
+        xi = torch.from_numpy(rng.standard_normal((rows, K)).astype(np.float32)).to(torch.bfloat16)
+        d = layer_desc(cu, su, cw, sw, xr.to(DEV), xi.to(DEV), N, K, rows)
+        st = status_word()
+        if gemm:
+            Q.ifq_gemm([d], T, rows, dev_status=st)
+        else:
+            run_gemv([d], T, rows, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cun, sun, cwn, swn,
+                      W.bf16_to_f32_numpy(xr), W.bf16_to_f32_numpy(xi))
