@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libifq.so")
-SOURCES = ["api.cu", "convert.cu", "quantize.cu", "dequantize.cu", "gemv.cu", "gemv_i8.cu", "gemv_fp4.cu", "gemm.cu", "product_generic.cu"]
+SOURCES = ["api.cu", "convert.cu", "quantize.cu", "dequantize.cu", "gemv.cu", "gemv_i8.cu", "gemm.cu", "product_generic.cu"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",

@@ -57,6 +57,33 @@ ifq_status check_qtensors(const ifq_qtensor* tensors, int count) {
   return IFQ_OK;
 }
 
+// Decode kernel for a call: CUDA cores for layers whose K is not a multiple of 64, else the integer
+// tensor-core kernel at one or two tokens and the bf16 kernel above them.
+enum class GemvPath : int32_t { kI8 = 0, kBf16 = 1, kGeneric = 2 };
+
+GemvPath gemv_path(const ifq_layer* L, int count, int B) {
+  if (ifq::any_narrow_k(L, count)) return GemvPath::kGeneric;
+  if (B <= ifq::IFQ_I8_MAX_BATCH) return GemvPath::kI8;
+  return GemvPath::kBf16;
+}
+
+size_t gemv_workspace(GemvPath path, const ifq_layer* L, int count, int T, int B) {
+  switch (path) {
+    case GemvPath::kI8: return ifq::gemv_i8_workspace_bytes(L, count, T, B);
+    case GemvPath::kBf16: return ifq::gemv_bf16_workspace_bytes(L, count, B);
+    default: return 0;
+  }
+}
+
+cudaError_t launch_path(GemvPath path, const ifq_layer* L, int count, int T, int B, void* ws, uint32_t* dev_status,
+                        cudaStream_t s) {
+  switch (path) {
+    case GemvPath::kI8: return ifq::launch_gemv_i8(L, count, T, B, ws, dev_status, s);
+    case GemvPath::kBf16: return ifq::launch_gemv(L, count, T, B, ws, dev_status, s);
+    default: return ifq::launch_product_generic(L, count, T, B, dev_status, s);
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -219,9 +246,7 @@ ifq_status ifq_dequantize(const ifq_dqtensor* tensors, int count, int T, ifq_str
 
 size_t ifq_gemv_workspace_bytes(const ifq_layer* layers, int count, int T, int B) {
   if (check_layers(layers, count, T) != IFQ_OK || B < 1 || B > IFQ_MAX_GEMV_BATCH) return 0;
-  if (ifq::any_narrow_k(layers, count)) return 0;
-  return B <= ifq::IFQ_FP4_MAX_BATCH ? ifq::gemv_fp4_workspace_bytes(layers, count, T, B)
-                                     : ifq::gemv_bf16_workspace_bytes(layers, count, B);
+  return gemv_workspace(gemv_path(layers, count, B), layers, count, T, B);
 }
 
 ifq_status ifq_gemv(const ifq_layer* layers, int count, int T, int B, void* workspace, size_t workspace_bytes,
@@ -229,38 +254,31 @@ ifq_status ifq_gemv(const ifq_layer* layers, int count, int T, int B, void* work
   ifq_status st = check_layers(layers, count, T);
   if (st != IFQ_OK) return st;
   if (B < 1 || B > IFQ_MAX_GEMV_BATCH) return IFQ_ERR_BATCH;
-  if (ifq::any_narrow_k(layers, count)) {
-    st = check_device();
-    if (st != IFQ_OK) return st;
-    return from_cuda(ifq::launch_product_generic(layers, count, T, B, dev_status, as_stream(stream)));
-  }
-  const bool fp4 = B <= ifq::IFQ_FP4_MAX_BATCH;
-  const size_t need = fp4 ? ifq::gemv_fp4_workspace_bytes(layers, count, T, B)
-                          : ifq::gemv_bf16_workspace_bytes(layers, count, B);
+  const GemvPath path = gemv_path(layers, count, B);
+  const size_t need = gemv_workspace(path, layers, count, T, B);
   if (need > 0 && (!workspace || workspace_bytes < need)) return IFQ_ERR_WORKSPACE;
   if (need > 0 && !aligned16(workspace)) return IFQ_ERR_ALIGN;
   st = check_device();
   if (st != IFQ_OK) return st;
-  if (fp4) return from_cuda(ifq::launch_gemv_fp4(layers, count, T, B, workspace, dev_status, as_stream(stream)));
-  return from_cuda(ifq::launch_gemv(layers, count, T, B, workspace, dev_status, as_stream(stream)));
+  return from_cuda(launch_path(path, layers, count, T, B, workspace, dev_status, as_stream(stream)));
 }
 
-// A prepared decode call, in the caller's host buffer: the routing and the descriptors, then (4-bit
+// A prepared decode call, in the caller's host buffer: the routing and the descriptors, then (integer
 // path) the finished launch parameters at a 64-byte boundary.
 namespace {
 constexpr uint32_t kPlanMagic = 0x50514649u;
 struct alignas(64) GemvPlanHeader {
   uint32_t magic;
-  int32_t path;  // 0: 4-bit tensor cores, 1: bf16 mma.sync, 2: CUDA cores (narrow K)
+  int32_t path;  // a GemvPath
   int32_t count, T, B;
   void* workspace;
   uint32_t* dev_status;
   ifq_layer layers[IFQ_MAX_GROUP];
 };
-constexpr size_t kPlanFp4Offset = (sizeof(GemvPlanHeader) + 63) & ~(size_t)63;
+constexpr size_t kPlanParamsOffset = (sizeof(GemvPlanHeader) + 63) & ~(size_t)63;
 }  // namespace
 
-size_t ifq_gemv_plan_bytes(void) { return kPlanFp4Offset + ifq::gemv_fp4_plan_bytes(); }
+size_t ifq_gemv_plan_bytes(void) { return kPlanParamsOffset + ifq::gemv_i8_plan_bytes(); }
 
 ifq_status ifq_gemv_prepare(const ifq_layer* layers, int count, int T, int B, void* workspace,
                             size_t workspace_bytes, uint32_t* dev_status, void* plan, size_t plan_bytes) {
@@ -270,27 +288,24 @@ ifq_status ifq_gemv_prepare(const ifq_layer* layers, int count, int T, int B, vo
   if (!plan) return IFQ_ERR_NULL;
   if (plan_bytes < ifq_gemv_plan_bytes()) return IFQ_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(plan) & 63u) return IFQ_ERR_ALIGN;
-  const bool narrow = ifq::any_narrow_k(layers, count);
-  const bool fp4 = !narrow && B <= ifq::IFQ_FP4_MAX_BATCH;
-  const size_t need = narrow ? 0
-                      : fp4  ? ifq::gemv_fp4_workspace_bytes(layers, count, T, B)
-                             : ifq::gemv_bf16_workspace_bytes(layers, count, B);
+  const GemvPath path = gemv_path(layers, count, B);
+  const size_t need = gemv_workspace(path, layers, count, T, B);
   if (need > 0 && (!workspace || workspace_bytes < need)) return IFQ_ERR_WORKSPACE;
   if (need > 0 && !aligned16(workspace)) return IFQ_ERR_ALIGN;
   st = check_device();
   if (st != IFQ_OK) return st;
   GemvPlanHeader* h = static_cast<GemvPlanHeader*>(plan);
   memset(h, 0, sizeof(GemvPlanHeader));
-  h->path = narrow ? 2 : fp4 ? 0 : 1;
+  h->path = (int32_t)path;
   h->count = count;
   h->T = T;
   h->B = B;
   h->workspace = workspace;
   h->dev_status = dev_status;
   memcpy(h->layers, layers, sizeof(ifq_layer) * count);
-  if (fp4) {
-    const cudaError_t e = ifq::plan_gemv_fp4(layers, count, T, B, workspace, dev_status,
-                                             static_cast<char*>(plan) + kPlanFp4Offset);
+  if (path == GemvPath::kI8) {
+    const cudaError_t e = ifq::plan_gemv_i8(layers, count, T, B, workspace, dev_status,
+                                             static_cast<char*>(plan) + kPlanParamsOffset);
     if (e != cudaSuccess) return IFQ_ERR_CUDA;
   }
   h->magic = kPlanMagic;
@@ -302,13 +317,10 @@ ifq_status ifq_gemv_run(const void* plan, ifq_stream_t stream) {
   if (reinterpret_cast<uintptr_t>(plan) & 63u) return IFQ_ERR_ALIGN;
   const GemvPlanHeader* h = static_cast<const GemvPlanHeader*>(plan);
   if (h->magic != kPlanMagic) return IFQ_ERR_NULL;
-  switch (h->path) {
-    case 0: return from_cuda(ifq::run_gemv_fp4_plan(static_cast<const char*>(plan) + kPlanFp4Offset, as_stream(stream)));
-    case 1:
-      return from_cuda(ifq::launch_gemv(h->layers, h->count, h->T, h->B, h->workspace, h->dev_status, as_stream(stream)));
-    default:
-      return from_cuda(ifq::launch_product_generic(h->layers, h->count, h->T, h->B, h->dev_status, as_stream(stream)));
-  }
+  const GemvPath path = (GemvPath)h->path;
+  if (path == GemvPath::kI8)
+    return from_cuda(ifq::run_gemv_i8_plan(static_cast<const char*>(plan) + kPlanParamsOffset, as_stream(stream)));
+  return from_cuda(launch_path(path, h->layers, h->count, h->T, h->B, h->workspace, h->dev_status, as_stream(stream)));
 }
 
 ifq_status ifq_gemm_wait_limit(const ifq_layer* layers, int count, int T, int64_t M, uint64_t wait_limit_ns,

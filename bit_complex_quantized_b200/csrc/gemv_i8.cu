@@ -816,15 +816,21 @@ size_t gemv_i8_workspace_bytes(const ifq_layer* Ls, int count, int T, int B) {
 namespace {
 
 template <int kCap, int NB>
-cudaError_t launch_cap(const ifq_layer* Ls, int count, int T, int B, void* ws, uint32_t* dev_status, cudaStream_t s) {
-  using P = I8Params<kCap>;
+cudaError_t kernel_attr() {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(gemv_i8_kernel<P, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMainSmem);
+    attr_err = cudaFuncSetAttribute(gemv_i8_kernel<I8Params<kCap>, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kMainSmem);
   });
-  if (attr_err != cudaSuccess) return attr_err;
-  P p;
+  return attr_err;
+}
+
+// The launch parameters of one call: the layers' descriptors and workspace slices, the tensor maps
+// of the codes, the prep grid and the main grid.
+template <int kCap, int NB>
+cudaError_t build_params(const ifq_layer* Ls, int count, int T, int B, void* ws, uint32_t* dev_status,
+                         I8Params<kCap>& p, int64_t& preps, int64_t& ctas) {
   memset(&p, 0, sizeof(p));
   p.count = count;
   p.T = T;
@@ -833,7 +839,8 @@ cudaError_t launch_cap(const ifq_layer* Ls, int count, int T, int B, void* ws, u
   WsLayout lay[IFQ_MAX_GROUP];
   layout_layers(Ls, count, T, NB, lay);
   char* base = static_cast<char*>(ws);
-  int64_t chunks = 0, preps = 0;
+  int64_t chunks = 0;
+  preps = 0;
   for (int i = 0; i < count; ++i) {
     I8Layer& a = p.L[i];
     a.codes[0] = Ls[i].codes_u;
@@ -876,18 +883,24 @@ cudaError_t launch_cap(const ifq_layer* Ls, int count, int T, int B, void* ws, u
   }
   p.total_chunks = chunks;
   if (chunks >= ((int64_t)1 << 40) || preps > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-
-  gemv_prep_kernel<P, NB><<<(unsigned)preps, kPrepThreads, 0, s>>>(p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-
   int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int64_t ctas = (int64_t)sms * ctas_per_sm(NB);
+  ctas = (int64_t)sms * ctas_per_sm(NB);
   const int64_t need = (chunks + kWarps - 1) / kWarps;  // at least one chunk per warp
   if (ctas > need) ctas = need;
   p.sms = ctas == (int64_t)sms * ctas_per_sm(NB) ? sms : 0;
+  return cudaSuccess;
+}
+
+// The prep kernel, then the main kernel as its programmatic dependent.
+template <int kCap, int NB>
+cudaError_t launch_params(const I8Params<kCap>& p, int64_t preps, int64_t ctas, cudaStream_t s) {
+  cudaError_t e = kernel_attr<kCap, NB>();
+  if (e != cudaSuccess) return e;
+  gemv_prep_kernel<I8Params<kCap>, NB><<<(unsigned)preps, kPrepThreads, 0, s>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3((unsigned)ctas);
@@ -899,7 +912,40 @@ cudaError_t launch_cap(const ifq_layer* Ls, int count, int T, int B, void* ws, u
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_i8_kernel<P, NB>, p);
+  return cudaLaunchKernelEx(&cfg, gemv_i8_kernel<I8Params<kCap>, NB>, p);
+}
+
+template <int kCap, int NB>
+cudaError_t launch_cap(const ifq_layer* Ls, int count, int T, int B, void* ws, uint32_t* dev_status, cudaStream_t s) {
+  I8Params<kCap> p;
+  int64_t preps = 0, ctas = 0;
+  const cudaError_t e = build_params<kCap, NB>(Ls, count, T, B, ws, dev_status, p, preps, ctas);
+  if (e != cudaSuccess) return e;
+  return launch_params<kCap, NB>(p, preps, ctas, s);
+}
+
+// A prepared call: the finished parameters of the largest group, reused by every run.
+struct alignas(64) I8Plan {
+  int32_t nb, cap;
+  int64_t preps, ctas;
+  alignas(64) unsigned char params[sizeof(I8Params<IFQ_MAX_GROUP>)];
+};
+
+template <int NB>
+cudaError_t plan_nb(const ifq_layer* Ls, int count, int T, int B, void* ws, uint32_t* st, I8Plan& pl) {
+  pl.nb = NB;
+  pl.cap = count <= 8 ? 8 : IFQ_MAX_GROUP;
+  if (pl.cap == 8)
+    return build_params<8, NB>(Ls, count, T, B, ws, st, *reinterpret_cast<I8Params<8>*>(pl.params), pl.preps, pl.ctas);
+  return build_params<IFQ_MAX_GROUP, NB>(Ls, count, T, B, ws, st,
+                                         *reinterpret_cast<I8Params<IFQ_MAX_GROUP>*>(pl.params), pl.preps, pl.ctas);
+}
+
+template <int NB>
+cudaError_t run_nb(const I8Plan& pl, cudaStream_t s) {
+  if (pl.cap == 8) return launch_params<8, NB>(*reinterpret_cast<const I8Params<8>*>(pl.params), pl.preps, pl.ctas, s);
+  return launch_params<IFQ_MAX_GROUP, NB>(*reinterpret_cast<const I8Params<IFQ_MAX_GROUP>*>(pl.params), pl.preps,
+                                          pl.ctas, s);
 }
 
 }  // namespace
@@ -914,6 +960,23 @@ cudaError_t launch_gemv_i8(const ifq_layer* Ls, int count, int T, int B, void* w
                            cudaStream_t s) {
   return gemv_i8_tokens(B) == 1 ? launch_nb<1>(Ls, count, T, B, ws, dev_status, s)
                                 : launch_nb<2>(Ls, count, T, B, ws, dev_status, s);
+}
+
+size_t gemv_i8_plan_bytes() { return sizeof(I8Plan); }
+
+cudaError_t plan_gemv_i8(const ifq_layer* Ls, int count, int T, int B, void* ws, uint32_t* dev_status, void* dst) {
+  I8Plan& pl = *static_cast<I8Plan*>(dst);
+  return gemv_i8_tokens(B) == 1 ? plan_nb<1>(Ls, count, T, B, ws, dev_status, pl)
+                                : plan_nb<2>(Ls, count, T, B, ws, dev_status, pl);
+}
+
+cudaError_t run_gemv_i8_plan(const void* src, cudaStream_t s) {
+  const I8Plan& pl = *static_cast<const I8Plan*>(src);
+  switch (pl.nb) {
+    case 1: return run_nb<1>(pl, s);
+    case 2: return run_nb<2>(pl, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace ifq

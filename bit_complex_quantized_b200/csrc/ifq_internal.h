@@ -39,22 +39,15 @@ size_t gemv_bf16_workspace_bytes(const ifq_layer* L, int count, int B);
 cudaError_t launch_gemv(const ifq_layer* L, int count, int T, int B, void* ws, uint32_t* dev_status,
                         cudaStream_t s);
 
-// Block-scaled 4-bit tensor-core path for B <= IFQ_FP4_MAX_BATCH tokens (gemv_fp4.cu): workspace size
-// (activation digits and factors, block tickets, per-unit partial slots) and launch.
-constexpr int IFQ_FP4_MAX_BATCH = 4;
-// A prepared call of the 4-bit path: its parameter block in a caller buffer (64-byte aligned).
-size_t gemv_fp4_plan_bytes();
-cudaError_t plan_gemv_fp4(const ifq_layer* L, int count, int T, int B, void* ws, uint32_t* dev_status, void* dst);
-cudaError_t run_gemv_fp4_plan(const void* src, cudaStream_t s);
-size_t gemv_fp4_workspace_bytes(const ifq_layer* L, int count, int T, int B);
-cudaError_t launch_gemv_fp4(const ifq_layer* L, int count, int T, int B, void* ws, uint32_t* dev_status,
-                            cudaStream_t s);
-
 // Integer tensor-core path for B <= IFQ_I8_MAX_BATCH tokens (gemv_i8.cu) and its workspace size.
 constexpr int IFQ_I8_MAX_BATCH = 2;
 size_t gemv_i8_workspace_bytes(const ifq_layer* L, int count, int T, int B);
 cudaError_t launch_gemv_i8(const ifq_layer* L, int count, int T, int B, void* ws, uint32_t* dev_status,
                            cudaStream_t s);
+// A prepared call of the integer path: its finished launch parameters in a caller buffer (64-byte aligned).
+size_t gemv_i8_plan_bytes();
+cudaError_t plan_gemv_i8(const ifq_layer* L, int count, int T, int B, void* ws, uint32_t* dev_status, void* dst);
+cudaError_t run_gemv_i8_plan(const void* src, cudaStream_t s);
 
 // Layers whose K is a multiple of 4 but not of 64 (product_generic.cu): any number of rows.
 cudaError_t launch_product_generic(const ifq_layer* L, int count, int T, int64_t rows, uint32_t* dev_status,

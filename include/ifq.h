@@ -363,8 +363,8 @@ ifq_status ifq_gemv(const ifq_layer* layers, int count, int T, int B, void* work
                     uint32_t* dev_status, ifq_stream_t stream);
 
 /* Prepared decode calls, for a caller that repeats the same call (a decode loop): ifq_gemv_prepare
- * validates the arguments and stores everything the launches need -- the routing, and for the 4-bit
- * tensor-core path the finished kernel parameters with their tensor maps -- in a caller-owned HOST
+ * validates the arguments and stores everything the launches need -- the routing, and for the integer
+ * tensor-core path (B <= 2) the finished kernel parameters with their tensor maps -- in a caller-owned HOST
  * buffer of ifq_gemv_plan_bytes() bytes, 64-byte aligned; ifq_gemv_run(plan, stream) then only
  * launches, and gives the same outputs as ifq_gemv with the same arguments.  Every tensor named by
  * the layers, the workspace and dev_status must stay allocated and in place while the plan is used

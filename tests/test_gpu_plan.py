@@ -1,5 +1,5 @@
 """Prepared decode calls: ifq_gemv_prepare + ifq_gemv_run give the outputs of ifq_gemv bit for bit on
-each path (4-bit tensor cores, bf16 mma.sync, CUDA cores for a narrow width), also after new
+each path (integer tensor cores at B <= 2, bf16 mma.sync above, CUDA cores for a narrow width), also after new
 activations are written into the same buffers between runs."""
 import numpy as np
 import pytest
@@ -18,7 +18,7 @@ def _cuda():
     Q.load()
 
 
-@pytest.mark.parametrize("B,K", [(1, 2048), (3, 1088), (8, 2048), (2, 100)])
+@pytest.mark.parametrize("B,K", [(1, 2048), (2, 4160), (3, 1088), (8, 2048), (2, 100)])
 def test_prepared_call_equals_ifq_gemv(B, K):
     rng = np.random.default_rng(B * 7 + K)
     N, T = 200, 2
