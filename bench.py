@@ -679,8 +679,20 @@ def e2e_decode(block, steps, warmup):
         if i >= warmup:
             times.append(a.elapsed_time(b) * 1e-3)
     t = statistics.mean(times)
+    # the same two copies with no kernel between them: the floor that the copies alone set
+    copies = []
+    for i in range(warmup + steps):
+        block.flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        x_dev.copy_(x_host, non_blocking=True)
+        y_host.copy_(y_dev, non_blocking=True)
+        b.record()
+        torch.cuda.synchronize()
+        if i >= warmup:
+            copies.append(a.elapsed_time(b) * 1e-3)
     return {"value": block.gemv_bytes(block.B) / t / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": t * 1e3}
+            "d2h_bytes_per_step": d2h, "ms_per_step": t * 1e3, "copies_only_ms": statistics.mean(copies) * 1e3}
 
 
 def max_over_ranks(values, device):
