@@ -21,12 +21,17 @@
 // (activations in by TMA and out to the tensor core, 16 KB per K16 step), so
 // the MMA is not starved by shared-memory bandwidth.
 //
+// One persistent launch per call: one CTA per SM walks a static list of the call's tiles (all
+// layers, longest K first), so the tail of one layer's tiles is filled by the next layer's, and the
+// copy / expansion / MMA pipeline and the TMEM allocation carry over from tile to tile; while the
+// epilogue stores one tile's y, the MMAs of the next tile run.
 // CTA tile: 128 tokens x 64 outputs; K in blocks of 64.  Warp roles (14 warps):
 //   0-3   expanders: code tile -> A rows in TMEM (warp w writes lanes 32w..32w+31;
 //         lane 32w + j holds output 16w + (j & 15), class Br for j < 16, Bi else)
 //   4-11  epilogue: tcgen05.ld of the finished (stage, branch) accumulator, the
 //         Br/Bi exchange between lanes j and j ^ 16, scales, and y accumulated
-//         in shared memory; y stored to global at the end
+//         in shared memory (the first pass of a tile overwrites it); y stored to
+//         global at the tile's end
 //   12    TMA producer: X_re, X_im tiles (128 B swizzle) and the 64 x 16-byte code tile
 //   13    TMEM allocator and single-thread MMA issuer (M=128, N=256, K=16 per instruction)
 // TMEM: the accumulator (256 columns) and 4 stages of A (32 columns each).
@@ -62,17 +67,34 @@ constexpr uint32_t kAcol = 2 * BM;              // A stage s at columns kAcol + 
 constexpr uint32_t kIdesc = umma_idesc_bf16(2 * BN, 2 * BM);
 static_assert(kAcol + STAGES * (BK / 2) <= kTmemCols, "TMEM budget");
 
-struct __align__(64) GemmArgs {
+// One layer of a grouped call.  Its output tiles are numbered from tile_begin: token tile
+// (128 tokens) major, output tile (64 outputs) minor, so that the tiles running at the same time
+// share their activation tiles in L2.
+struct __align__(64) GemmLayer {
   CUtensorMap tmap_x[2];      // bf16 [M][K]: box {64, 128}, 128 B swizzle
   CUtensorMap tmap_codes[2];  // u8 [T*N][K/4]: box {16, 64}
   const float* scales[2];
   float* y[2];
-  const float* rot[2];  // optional epilogue rotation [M][N] (re, im), or null
-  int64_t N, K, M;
-  int T, nbranch;
-  uint64_t wait_ns;  // limit of each pipeline wait (drains after a lost wait keep IFQ_WAIT_LIMIT_NS)
-  uint32_t* status;
+  const float* rot[2];        // optional epilogue rotation [M][N] (re, im), or null
+  int64_t N, K;
+  int64_t tile_begin;
+  int32_t nbranch, tiles_n;
 };
+
+// Capacity kCap >= count.  The layers are stored heaviest first (most K steps per tile), so that the
+// CTAs take the long tiles before the short ones.
+template <int kCap>
+struct __align__(64) GemmParams {
+  int64_t tile_begin[kCap];   // copies of the layers' first tiles, for the tile -> layer search
+  int64_t tiles;              // all tiles of the call
+  int64_t M;
+  int count, T;
+  uint64_t wait_ns;           // limit of each pipeline wait (drains after a lost wait keep IFQ_WAIT_LIMIT_NS)
+  uint32_t* status;
+  GemmLayer L[kCap];
+};
+
+static_assert(sizeof(GemmParams<IFQ_MAX_GROUP>) <= 32764, "kernel parameter block limit");
 
 struct Smem {
   uint64_t full_tma[STAGES];
@@ -83,7 +105,26 @@ struct Smem {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  int epi_stop;
 };
+
+struct Tile {
+  int li;
+  int64_t n0, m0;
+};
+
+template <int kCap>
+__device__ __forceinline__ Tile decode_tile(const GemmParams<kCap>& p, int64_t t) {
+  int li = 0;
+  while (li + 1 < p.count && t >= p.tile_begin[li + 1]) ++li;
+  const int64_t local = t - p.tile_begin[li];
+  const int64_t tn = p.L[li].tiles_n;
+  Tile r;
+  r.li = li;
+  r.n0 = (local % tn) * BN;
+  r.m0 = (local / tn) * BM;
+  return r;
+}
 
 // Two codes (bits 0..3 of `nib`) -> one 32-bit column of A: the bf16 pair (Br or Bi of the
 // lower code in the low half).  The multiply places code 0's axis bit on bit 14 (the exponent
@@ -95,7 +136,57 @@ __device__ __forceinline__ uint32_t expand_pair(uint32_t nib, bool imag) {
   return imag ? spread : spread ^ 0x40004000u;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ GemmArgs a) {
+// Store a finished tile's y from shared memory ([plane][token][output]), rows of 64 outputs as float4,
+// with the optional rotation.  e: the calling thread's index among the 256 epilogue threads.
+__device__ __forceinline__ void store_tile_y(const GemmLayer& L, int64_t M, const Tile& tl, const float* ys, int e) {
+  const bool vec = (L.N & 3) == 0 && tl.n0 + BN <= L.N;
+  for (int idx = e; idx < BM * (BN / 4); idx += kEpiWarps * 32) {
+    const int tok = idx / (BN / 4), c4 = idx - tok * (BN / 4);
+    const int64_t m = tl.m0 + tok;
+    if (m >= M) continue;
+    const float4 r4 = *reinterpret_cast<const float4*>(ys + tok * BN + 4 * c4);
+    const float4 i4 = *reinterpret_cast<const float4*>(ys + BM * BN + tok * BN + 4 * c4);
+    float vr[4] = {r4.x, r4.y, r4.z, r4.w}, vi[4] = {i4.x, i4.y, i4.z, i4.w};
+    const int64_t o = m * L.N + tl.n0 + 4 * c4;
+    const int nv = vec ? 4 : (int)(L.N - (tl.n0 + 4 * c4) < 4 ? L.N - (tl.n0 + 4 * c4) : 4);  // valid outputs
+    if (L.rot[0]) {  // complex RoPE: times rot[m][n]
+      float cr[4] = {1.f, 1.f, 1.f, 1.f}, ci[4] = {0.f, 0.f, 0.f, 0.f};
+      if (vec) {
+        const float4 c = __ldg(reinterpret_cast<const float4*>(L.rot[0] + o));
+        const float4 d = __ldg(reinterpret_cast<const float4*>(L.rot[1] + o));
+        cr[0] = c.x; cr[1] = c.y; cr[2] = c.z; cr[3] = c.w;
+        ci[0] = d.x; ci[1] = d.y; ci[2] = d.z; ci[3] = d.w;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (j < nv) {
+            cr[j] = __ldg(L.rot[0] + o + j);
+            ci[j] = __ldg(L.rot[1] + o + j);
+          }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float r = cr[j] * vr[j] - ci[j] * vi[j], im = cr[j] * vi[j] + ci[j] * vr[j];
+        vr[j] = r;
+        vi[j] = im;
+      }
+    }
+    if (vec) {
+      *reinterpret_cast<float4*>(L.y[0] + o) = make_float4(vr[0], vr[1], vr[2], vr[3]);
+      *reinterpret_cast<float4*>(L.y[1] + o) = make_float4(vi[0], vi[1], vi[2], vi[3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (j < nv) {
+          L.y[0][o + j] = vr[j];
+          L.y[1][o + j] = vi[j];
+        }
+    }
+  }
+}
+
+template <int kCap>
+__global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ GemmParams<kCap> p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* ys = reinterpret_cast<float*>(smem + STAGES * kStageBytes);
@@ -103,10 +194,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   volatile int* abort = &S->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t n0 = (int64_t)blockIdx.x * BN;
-  const int64_t m0 = (int64_t)blockIdx.y * BM;
-  const int KB = (int)(a.K / BK);
-  const int P = a.T * a.nbranch;
+  const int P = p.T;  // passes per tile: T stages x the layer's branches (times nbranch below)
+  const int64_t t_first = blockIdx.x, t_step = gridDim.x;
 
   auto xtile = [&](int s) { return smem + s * kStageBytes; };  // X_re, then X_im 16 KB later
   auto ctile = [&](int s) { return smem + s * kStageBytes + 2 * kTileX; };
@@ -121,13 +210,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     mbar_init(&S->acc_empty, kEpiWarps);
     mbar_init(&S->drain, 1);
     S->abort = 0;
+    S->epi_stop = 0;
     fence_mbar_init();
-    prefetch_tmap(&a.tmap_x[0]);
-    prefetch_tmap(&a.tmap_x[1]);
-    prefetch_tmap(&a.tmap_codes[0]);
-    if (a.nbranch > 1) prefetch_tmap(&a.tmap_codes[1]);
   }
-  for (uint32_t i = threadIdx.x; i < kYFloats; i += kThreads) ys[i] = 0.0f;
+  if (warp == kProducerWarp && lane < p.count) {
+    const GemmLayer& L = p.L[lane];
+    prefetch_tmap(&L.tmap_x[0]);
+    prefetch_tmap(&L.tmap_x[1]);
+    prefetch_tmap(&L.tmap_codes[0]);
+    if (L.nbranch > 1) prefetch_tmap(&L.tmap_codes[1]);
+  }
   if (warp == kMmaWarp) {
     tmem_alloc(&S->tmem_base, kTmemCols);
     tmem_relinquish();
@@ -142,19 +234,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     if (lane == 0) {
       int issued[STAGES];
       for (int s = 0; s < STAGES; ++s) issued[s] = 0;
-      for (int p = 0; p < P && !*abort; ++p) {
-        const int t = p / a.nbranch, br = p % a.nbranch;
-        const int32_t crow = (int32_t)((int64_t)t * a.N + n0);
-        for (int kb = 0; kb < KB; ++kb) {
-          const int it = p * KB + kb, s = it % STAGES;
-          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!mbar_wait_bounded_ns(&S->empty[s], ph ^ 1u, abort, a.wait_ns)) break;
-          mbar_arrive_expect_tx(&S->full_tma[s], kTmaBytes);
-          tma_load_2d(xtile(s), &a.tmap_x[0], kb * BK, (int32_t)m0, &S->full_tma[s]);
-          tma_load_2d(xtile(s) + kTileX, &a.tmap_x[1], kb * BK, (int32_t)m0, &S->full_tma[s]);
-          tma_load_2d(ctile(s), &a.tmap_codes[br], kb * (BK / 4), crow, &S->full_tma[s]);
-          ++issued[s];
+      int it = 0;  // stage fills of this CTA, across its tiles
+      for (int64_t tt = t_first; tt < p.tiles && !*abort; tt += t_step) {
+        const Tile tl = decode_tile(p, tt);
+        const GemmLayer& L = p.L[tl.li];
+        const int KB = (int)(L.K / BK), np = P * L.nbranch;
+        bool ok = true;
+        for (int q = 0; q < np && ok; ++q) {
+          const int t = q / L.nbranch, br = q % L.nbranch;
+          const int32_t crow = (int32_t)((int64_t)t * L.N + tl.n0);
+          for (int kb = 0; kb < KB; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+            if (!mbar_wait_bounded_ns(&S->empty[s], ph ^ 1u, abort, p.wait_ns)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&S->full_tma[s], kTmaBytes);
+            tma_load_2d(xtile(s), &L.tmap_x[0], kb * BK, (int32_t)tl.m0, &S->full_tma[s]);
+            tma_load_2d(xtile(s) + kTileX, &L.tmap_x[1], kb * BK, (int32_t)tl.m0, &S->full_tma[s]);
+            tma_load_2d(ctile(s), &L.tmap_codes[br], kb * (BK / 4), crow, &S->full_tma[s]);
+            ++issued[s];
+          }
         }
+        if (!ok) break;
       }
       if (*abort) {
         // Let every issued copy land before the CTA's shared memory is released.
@@ -166,30 +269,37 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer (whole warp, one elected lane issues)
     const uint64_t xdesc0 = umma_desc_sw128(smem_u32(xtile(0)));
-    for (int p = 0; p < P; ++p) {
-      // the epilogue has read the previous (stage, branch) accumulator
-      int ok = 1;
-      if (lane == 0) ok = !*abort && mbar_wait_bounded_ns(&S->acc_empty, ((uint32_t)p & 1u) ^ 1u, abort, a.wait_ns);
-      ok = __shfl_sync(0xffffffffu, ok, 0);  // every lane takes lane 0's result: the warp stays converged
-      if (!ok) break;
-      tc_fence_after();
-      for (int kb = 0; kb < KB; ++kb) {
-        const int it = p * KB + kb, s = it % STAGES;
-        const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-        if (lane == 0)
-          ok = mbar_wait_bounded_ns(&S->full_tma[s], ph, abort, a.wait_ns) &&
-               mbar_wait_bounded_ns(&S->full_a[s], ph, abort, a.wait_ns);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+    int it = 0, gp = 0;  // stage uses and (stage, branch) passes of this CTA, across its tiles
+    bool ok = true;
+    for (int64_t tt = t_first; tt < p.tiles && ok; tt += t_step) {
+      const Tile tl = decode_tile(p, tt);
+      const GemmLayer& L = p.L[tl.li];
+      const int KB = (int)(L.K / BK), np = P * L.nbranch;
+      for (int q = 0; q < np && ok; ++q, ++gp) {
+        // the epilogue has read the previous pass's accumulator
+        int w_ok = 1;
+        if (lane == 0) w_ok = !*abort && mbar_wait_bounded_ns(&S->acc_empty, ((uint32_t)gp & 1u) ^ 1u, abort, p.wait_ns);
+        ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0;  // every lane takes lane 0's result: the warp stays converged
         if (!ok) break;
         tc_fence_after();
-        // the four K16 steps of the stage: B advances 32 bytes (2 descriptor units) per step inside the
-        // 128-byte swizzle row, A 8 TMEM columns
-        umma_bf16_ta_x4(tmem, tmem + kAcol + 32 * s, xdesc0 + (uint64_t)((uint32_t)s * (kStageBytes >> 4)), kIdesc,
-                        kb != 0);
-        umma_commit_elect(&S->empty[s]);
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (lane == 0)
+            w_ok = mbar_wait_bounded_ns(&S->full_tma[s], ph, abort, p.wait_ns) &&
+                   mbar_wait_bounded_ns(&S->full_a[s], ph, abort, p.wait_ns);
+          ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0;
+          if (!ok) break;
+          tc_fence_after();
+          // the four K16 steps of the stage: B advances 32 bytes (2 descriptor units) per step inside the
+          // 128-byte swizzle row, A 8 TMEM columns
+          umma_bf16_ta_x4(tmem, tmem + kAcol + 32 * s, xdesc0 + (uint64_t)((uint32_t)s * (kStageBytes >> 4)), kIdesc,
+                          kb != 0);
+          umma_commit_elect(&S->empty[s]);
+        }
+        if (!ok) break;
+        umma_commit_elect(&S->acc_full);
       }
-      if (!ok) break;
-      umma_commit_elect(&S->acc_full);
     }
     if (lane == 0 && *abort) {
       volatile int never = 0;
@@ -201,140 +311,115 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     const bool imag = lane >= 16;
     const int o = 16 * warp + (lane & 15);   // this lane's output row within the tile
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16) + kAcol;
-    for (int p = 0; p < P && !__shfl_sync(0xffffffffu, *abort, 0); ++p) {
-      for (int kb = 0; kb < KB; ++kb) {
-        const int it = p * KB + kb, s = it % STAGES;
-        const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-        int ok = 1;
-        if (lane == 0)
-          ok = mbar_wait_bounded_ns(&S->empty[s], ph ^ 1u, abort, a.wait_ns) &&
-               mbar_wait_bounded_ns(&S->full_tma[s], ph, abort, a.wait_ns);
-        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-        // Rows past N carry other stages' or no codes; their outputs are never stored.
-        const uint4 cw = *reinterpret_cast<const uint4*>(ctile(s) + o * 16);
-        const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
-        uint32_t col[32];
+    int it = 0;
+    bool ok = true;
+    for (int64_t tt = t_first; tt < p.tiles && ok; tt += t_step) {
+      const Tile tl = decode_tile(p, tt);
+      const GemmLayer& L = p.L[tl.li];
+      const int KB = (int)(L.K / BK), np = P * L.nbranch;
+      for (int q = 0; q < np && ok; ++q) {
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          int w_ok = 1;
+          if (lane == 0)
+            w_ok = mbar_wait_bounded_ns(&S->empty[s], ph ^ 1u, abort, p.wait_ns) &&
+                   mbar_wait_bounded_ns(&S->full_tma[s], ph, abort, p.wait_ns);
+          ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0;
+          if (!ok) break;
+          // Rows past N carry other stages' or no codes; their outputs are never stored.
+          const uint4 cw = *reinterpret_cast<const uint4*>(ctile(s) + o * 16);
+          const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+          uint32_t col[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) col[c] = expand_pair((w[c >> 3] >> (4 * (c & 7))) & 0xFu, imag);
-        tmem_st_32x32b_x32(trow + 32 * s, col);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S->full_a[s]);
+          for (int c = 0; c < 32; ++c) col[c] = expand_pair((w[c >> 3] >> (4 * (c & 7))) & 0xFu, imag);
+          tmem_st_32x32b_x32(trow + 32 * s, col);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S->full_a[s]);
+        }
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;                  // TMEM lane quarter
+    const int qd = warp & 3;                   // TMEM lane quarter
     const int half = (warp - kExpWarps) >> 2;  // token chunks c with c % 2 == half
     const bool imag = lane >= 16;
-    const int o = 16 * q + (lane & 15);
-    const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-    for (int p = 0; p < P && !__shfl_sync(0xffffffffu, *abort, 0); ++p) {
-      int ok = 1;
-      if (lane == 0) ok = mbar_wait_bounded_ns(&S->acc_full, (uint32_t)p & 1u, abort, a.wait_ns);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      tc_fence_after();
-      const int t = p / a.nbranch, br = p % a.nbranch;
-      const float hr = 0.5f * __ldg(a.scales[br] + 2 * t);
-      const float hi = 0.5f * __ldg(a.scales[br] + 2 * t + 1);
-      const float sgn = br == 0 ? -1.0f : 1.0f;
+    const int o = 16 * qd + (lane & 15);
+    const uint32_t trow = tmem + ((uint32_t)(qd * 32) << 16);
+    const int e = threadIdx.x - kExpWarps * 32;  // 0..255
+    int gp = 0;
+    for (int64_t tt = t_first; tt < p.tiles; tt += t_step) {
+      const Tile tl = decode_tile(p, tt);
+      const GemmLayer& L = p.L[tl.li];
+      const int np = P * L.nbranch;
+      bool ok = true;
+      for (int q = 0; q < np; ++q, ++gp) {
+        int w_ok = 1;
+        if (lane == 0) w_ok = mbar_wait_bounded_ns(&S->acc_full, (uint32_t)gp & 1u, abort, p.wait_ns);
+        ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0;
+        if (!ok) break;
+        tc_fence_after();
+        const int t = q / L.nbranch, br = q % L.nbranch;
+        const float hr = 0.5f * __ldg(L.scales[br] + 2 * t);
+        const float hi = 0.5f * __ldg(L.scales[br] + 2 * t + 1);
+        const float sgn = br == 0 ? -1.0f : 1.0f;
 #pragma unroll 1
-      for (int c = half; c < BM / 32; c += 2) {
-        uint32_t u[32], v[32];
-        tmem_ld_32x32b_x32(trow + 32 * c, u);         // this lane's class, real plane, tokens 32c..
-        tmem_ld_32x32b_x32(trow + BM + 32 * c, v);    // imaginary plane
-        tmem_wait_ld();
-        // lane j < 16 (Br) takes tokens 32c + 0..15, lane j >= 16 (Bi) tokens 32c + 16..31;
-        // each gets the other class's values of its tokens from lane j ^ 16.  This lane's y
-        // entries are read first, then updated and written back, so the 16 read-add-write
-        // chains overlap.
-        const int tok0 = 32 * c + (imag ? 16 : 0);
-        float* yre = ys + tok0 * BN + o;
-        float* yim = ys + BM * BN + tok0 * BN + o;
-        float cre[16], cim[16];
+        for (int c = half; c < BM / 32; c += 2) {
+          uint32_t u[32], v[32];
+          tmem_ld_32x32b_x32(trow + 32 * c, u);         // this lane's class, real plane, tokens 32c..
+          tmem_ld_32x32b_x32(trow + BM + 32 * c, v);    // imaginary plane
+          tmem_wait_ld();
+          // lane j < 16 (Br) takes tokens 32c + 0..15, lane j >= 16 (Bi) tokens 32c + 16..31;
+          // each gets the other class's values of its tokens from lane j ^ 16.  The first pass of a
+          // tile writes this lane's y entries, the later ones read, update and write them back.
+          const int tok0 = 32 * c + (imag ? 16 : 0);
+          float* yre = ys + tok0 * BN + o;
+          float* yim = ys + BM * BN + tok0 * BN + o;
+          float cre[16], cim[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          cre[i] = yre[i * BN];
-          cim[i] = yim[i * BN];
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float mu_lo = __uint_as_float(u[i]), mv_lo = __uint_as_float(v[i]);
-          const float mu_hi = __uint_as_float(u[16 + i]), mv_hi = __uint_as_float(v[16 + i]);
-          // send the partner the values of the partner's tokens, receive those of mine
-          const float pu = __shfl_xor_sync(0xffffffffu, imag ? mu_lo : mu_hi, 16);
-          const float pv = __shfl_xor_sync(0xffffffffu, imag ? mv_lo : mv_hi, 16);
-          const float mu = imag ? mu_hi : mu_lo, mv = imag ? mv_hi : mv_lo;
-          const float P_rr = imag ? pu : mu, P_ri = imag ? pv : mv;
-          const float P_ir = imag ? mu : pu, P_ii = imag ? mv : pv;
-          cre[i] += hr * P_rr + sgn * hi * P_ii;
-          cim[i] += hi * P_ir - sgn * hr * P_ri;
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          yre[i * BN] = cre[i];
-          yim[i * BN] = cim[i];
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S->acc_empty);
-    }
-    // all epilogue warps have finished the tile's y: store it (rows of 64 outputs, float4)
-    asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
-    if (!__shfl_sync(0xffffffffu, *abort, 0)) {
-      const int e = threadIdx.x - kExpWarps * 32;  // 0..255
-      const bool vec = (a.N & 3) == 0 && n0 + BN <= a.N;
-      for (int idx = e; idx < BM * (BN / 4); idx += kEpiWarps * 32) {
-        const int tok = idx / (BN / 4), c4 = idx - tok * (BN / 4);
-        const int64_t m = m0 + tok;
-        if (m >= a.M) continue;
-        const float4 r4 = *reinterpret_cast<const float4*>(ys + tok * BN + 4 * c4);
-        const float4 i4 = *reinterpret_cast<const float4*>(ys + BM * BN + tok * BN + 4 * c4);
-        float vr[4] = {r4.x, r4.y, r4.z, r4.w}, vi[4] = {i4.x, i4.y, i4.z, i4.w};
-        const int64_t o = m * a.N + n0 + 4 * c4;
-        const int nv = vec ? 4 : (int)(a.N - (n0 + 4 * c4) < 4 ? a.N - (n0 + 4 * c4) : 4);  // valid outputs
-        if (a.rot[0]) {  // complex RoPE: times rot[m][n]
-          float cr[4] = {1.f, 1.f, 1.f, 1.f}, ci[4] = {0.f, 0.f, 0.f, 0.f};
-          if (vec) {
-            const float4 c = __ldg(reinterpret_cast<const float4*>(a.rot[0] + o));
-            const float4 d = __ldg(reinterpret_cast<const float4*>(a.rot[1] + o));
-            cr[0] = c.x; cr[1] = c.y; cr[2] = c.z; cr[3] = c.w;
-            ci[0] = d.x; ci[1] = d.y; ci[2] = d.z; ci[3] = d.w;
-          } else {
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              if (j < nv) {
-                cr[j] = __ldg(a.rot[0] + o + j);
-                ci[j] = __ldg(a.rot[1] + o + j);
-              }
+          for (int i = 0; i < 16; ++i) {
+            cre[i] = q == 0 ? 0.0f : yre[i * BN];
+            cim[i] = q == 0 ? 0.0f : yim[i * BN];
           }
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float r = cr[j] * vr[j] - ci[j] * vi[j], im = cr[j] * vi[j] + ci[j] * vr[j];
-            vr[j] = r;
-            vi[j] = im;
+          for (int i = 0; i < 16; ++i) {
+            const float mu_lo = __uint_as_float(u[i]), mv_lo = __uint_as_float(v[i]);
+            const float mu_hi = __uint_as_float(u[16 + i]), mv_hi = __uint_as_float(v[16 + i]);
+            // send the partner the values of the partner's tokens, receive those of mine
+            const float pu = __shfl_xor_sync(0xffffffffu, imag ? mu_lo : mu_hi, 16);
+            const float pv = __shfl_xor_sync(0xffffffffu, imag ? mv_lo : mv_hi, 16);
+            const float mu = imag ? mu_hi : mu_lo, mv = imag ? mv_hi : mv_lo;
+            const float P_rr = imag ? pu : mu, P_ri = imag ? pv : mv;
+            const float P_ir = imag ? mu : pu, P_ii = imag ? mv : pv;
+            cre[i] += hr * P_rr + sgn * hi * P_ii;
+            cim[i] += hi * P_ir - sgn * hr * P_ri;
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            yre[i * BN] = cre[i];
+            yim[i * BN] = cim[i];
           }
         }
-        if (vec) {
-          *reinterpret_cast<float4*>(a.y[0] + o) = make_float4(vr[0], vr[1], vr[2], vr[3]);
-          *reinterpret_cast<float4*>(a.y[1] + o) = make_float4(vi[0], vi[1], vi[2], vi[3]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (j < nv) {
-              a.y[0][o + j] = vr[j];
-              a.y[1][o + j] = vi[j];
-            }
-        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S->acc_empty);
       }
+      // The tile's y is complete in shared memory.  Every epilogue warp takes the same decision to go
+      // on (a lost wait anywhere stops them all at this point), then they store y together.
+      asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
+      if (e == 0) S->epi_stop = *abort;
+      asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
+      if (S->epi_stop) break;
+      store_tile_y(L, p.M, tl, ys, e);
+      asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");  // ys is free for the next tile
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0 && S->abort) set_status(a.status, IFQ_DEV_TIMEOUT);
+  if (threadIdx.x == 0 && S->abort) set_status(p.status, IFQ_DEV_TIMEOUT);
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -380,46 +465,77 @@ bool encode_tiled_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const vo
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-cudaError_t launch_gemm(const ifq_layer* Ls, int count, int T, int64_t M, uint64_t wait_ns, uint32_t* dev_status,
-                        cudaStream_t s) {
+namespace {
+
+template <int kCap>
+cudaError_t launch_cap(const ifq_layer* Ls, int count, int T, int64_t M, uint64_t wait_ns, uint32_t* dev_status,
+                       cudaStream_t s) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    attr_err = cudaFuncSetAttribute(gemm_kernel<kCap>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
+  GemmParams<kCap> p;
+  memset(&p, 0, sizeof(p));
+  p.count = count;
+  p.T = T;
+  p.M = M;
+  p.wait_ns = wait_ns;
+  p.status = dev_status;
+  // heaviest layers first: K steps per tile times (stage, branch) passes
+  int order[IFQ_MAX_GROUP];
+  for (int i = 0; i < count; ++i) order[i] = i;
+  for (int i = 1; i < count; ++i)
+    for (int j = i; j > 0; --j) {
+      const ifq_layer &a = Ls[order[j - 1]], &b = Ls[order[j]];
+      const int64_t wa = a.K * (a.codes_w ? 2 : 1), wb = b.K * (b.codes_w ? 2 : 1);
+      if (wa >= wb) break;
+      const int t = order[j - 1];
+      order[j - 1] = order[j];
+      order[j] = t;
+    }
+  const int64_t tiles_m = (M + BM - 1) / BM;
+  int64_t tiles = 0;
   for (int i = 0; i < count; ++i) {
-    const ifq_layer& L = Ls[i];
-    GemmArgs a;
-    memset(&a, 0, sizeof(a));
-    a.nbranch = L.codes_w ? 2 : 1;
-    a.N = L.N;
-    a.K = L.K;
-    a.M = M;
-    a.T = T;
-    a.status = dev_status;
-    a.wait_ns = wait_ns;
-    a.scales[0] = L.scales_u;
-    a.scales[1] = L.scales_w;
-    a.y[0] = L.y_re;
-    a.y[1] = L.y_im;
-    a.rot[0] = L.rot_re;
-    a.rot[1] = L.rot_im;
-    bool ok = make_map_2d(&a.tmap_x[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L.x_re, (uint64_t)L.K, (uint64_t)M,
+    const ifq_layer& L = Ls[order[i]];
+    GemmLayer& g = p.L[i];
+    g.nbranch = L.codes_w ? 2 : 1;
+    g.N = L.N;
+    g.K = L.K;
+    g.scales[0] = L.scales_u;
+    g.scales[1] = L.scales_w;
+    g.y[0] = L.y_re;
+    g.y[1] = L.y_im;
+    g.rot[0] = L.rot_re;
+    g.rot[1] = L.rot_im;
+    g.tiles_n = (int32_t)((L.N + BN - 1) / BN);
+    g.tile_begin = p.tile_begin[i] = tiles;
+    tiles += (int64_t)g.tiles_n * tiles_m;
+    bool ok = make_map_2d(&g.tmap_x[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L.x_re, (uint64_t)L.K, (uint64_t)M,
                           (uint64_t)L.K * 2, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              make_map_2d(&a.tmap_x[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L.x_im, (uint64_t)L.K, (uint64_t)M,
+              make_map_2d(&g.tmap_x[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L.x_im, (uint64_t)L.K, (uint64_t)M,
                           (uint64_t)L.K * 2, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B);
-    for (int b = 0; b < a.nbranch && ok; ++b)
-      ok = make_map_2d(&a.tmap_codes[b], CU_TENSOR_MAP_DATA_TYPE_UINT8, b == 0 ? L.codes_u : L.codes_w,
-                       (uint64_t)L.K / 4, (uint64_t)T * L.N, (uint64_t)L.K / 4, BK / 4, BN,
-                       CU_TENSOR_MAP_SWIZZLE_NONE);
+    for (int b = 0; b < g.nbranch && ok; ++b)
+      ok = make_map_2d(&g.tmap_codes[b], CU_TENSOR_MAP_DATA_TYPE_UINT8, b == 0 ? L.codes_u : L.codes_w,
+                       (uint64_t)L.K / 4, (uint64_t)T * L.N, (uint64_t)L.K / 4, BK / 4, BN, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return cudaErrorInvalidValue;
-    dim3 grid((unsigned)((L.N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
-    gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(a);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
   }
-  return cudaSuccess;
+  p.tiles = tiles;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t grid = tiles < sms ? tiles : sms;  // one persistent CTA per SM
+  gemm_kernel<kCap><<<(unsigned)grid, kThreads, kSmemBytes, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const ifq_layer* Ls, int count, int T, int64_t M, uint64_t wait_ns, uint32_t* dev_status,
+                        cudaStream_t s) {
+  return count <= 8 ? launch_cap<8>(Ls, count, T, M, wait_ns, dev_status, s)
+                    : launch_cap<IFQ_MAX_GROUP>(Ls, count, T, M, wait_ns, dev_status, s);
 }
 
 }  // namespace ifq

@@ -383,8 +383,9 @@ ifq_status ifq_gemv_run(const void* plan, ifq_stream_t stream);
  * codes are expanded straight into TMEM as exact {-2, 0, +2} bf16 operands (the
  * MMA's A operand), the +-1 and +-i classes accumulate in separate rows of a
  * float32 TMEM accumulator, and the scales are applied per (stage, branch) in
- * the epilogue.  Layers run one after
- * another on the stream.  dev_status may be NULL (timeouts then go unreported). */
+ * the epilogue.  All layers of the call run in one persistent launch (one CTA
+ * per SM over every layer's tiles, the layers with the longest K first).
+ * dev_status may be NULL (timeouts then go unreported). */
 ifq_status ifq_gemm(const ifq_layer* layers, int count, int T, int64_t M, uint32_t* dev_status,
                     ifq_stream_t stream);
 
