@@ -25,15 +25,18 @@
 // layers, longest K first), so the tail of one layer's tiles is filled by the next layer's, and the
 // copy / expansion / MMA pipeline and the TMEM allocation carry over from tile to tile; while the
 // epilogue stores one tile's y, the MMAs of the next tile run.
-// CTA tile: 128 tokens x 64 outputs; K in blocks of 64.  Warp roles (14 warps):
+// CTA tile: 128 tokens x 64 outputs; K in blocks of 64.  Warp roles (15 warps):
 //   0-3   expanders: code tile -> A rows in TMEM (warp w writes lanes 32w..32w+31;
 //         lane 32w + j holds output 16w + (j & 15), class Br for j < 16, Bi else)
 //   4-11  epilogue: tcgen05.ld of the finished (stage, branch) accumulator, the
 //         Br/Bi exchange between lanes j and j ^ 16, scales, and y accumulated
 //         in shared memory (the first pass of a tile overwrites it); y stored to
-//         global at the tile's end
-//   12    TMA producer: X_re, X_im tiles (128 B swizzle) and the 64 x 16-byte code tile
+//         global at the tile's end.  Each warp releases the accumulator right
+//         after its last TMEM read of the pass, before that chunk's arithmetic.
+//   12    TMA producer of the activations: X_re, X_im tiles (128 B swizzle), 4 stages
 //   13    TMEM allocator and single-thread MMA issuer (M=128, N=256, K=16 per instruction)
+//   14    TMA producer of the codes: 64 x 16-byte tiles in a ring of 16 stages of their own, so
+//         that an expander finds its codes in place as soon as its A stage is free
 // TMEM: the accumulator (256 columns) and 4 stages of A (32 columns each).
 // Every mbarrier wait is bounded; a lost wait sets IFQ_DEV_TIMEOUT, the CTA
 // drains its outstanding copies and MMAs, frees TMEM and returns.
@@ -50,18 +53,23 @@ namespace {
 constexpr int BM = 128;      // tokens per tile; the MMA's N is 2 BM (both planes)
 constexpr int BN = 64;       // outputs per tile; the MMA's M is 2 BN (Br and Bi rows)
 constexpr int BK = 64;       // K per stage (one 128-byte swizzle row of bf16)
-constexpr int STAGES = 4;
+constexpr int STAGES = 4;                    // activation stages in shared memory = A stages in TMEM
+constexpr int CSTAGES = 16;                  // code stages: a ring of its own, filled far ahead
 constexpr int kExpWarps = 4;
 constexpr int kEpiWarps = 8;                 // two per TMEM lane quarter, each half the tokens
 constexpr int kProducerWarp = kExpWarps + kEpiWarps;
 constexpr int kMmaWarp = kProducerWarp + 1;
-constexpr int kThreads = (kMmaWarp + 1) * 32;
+constexpr int kCodeWarp = kMmaWarp + 1;
+constexpr int kThreads = (kCodeWarp + 1) * 32;
 constexpr uint32_t kTileX = BM * BK * 2;        // 16 KB per activation plane
 constexpr uint32_t kTileC = BN * (BK / 4);      // 1 KB of codes
-constexpr uint32_t kStageBytes = 2 * kTileX + kTileC;  // 33 KB (multiple of 1 KB)
-constexpr uint32_t kTmaBytes = 2 * kTileX + kTileC;
+constexpr uint32_t kStageBytes = 2 * kTileX;    // 32 KB: X_re, X_im
+constexpr uint32_t kTmaBytes = 2 * kTileX;
+constexpr uint32_t kCodeOff = STAGES * kStageBytes;
+constexpr uint32_t kYOff = kCodeOff + CSTAGES * kTileC;
 constexpr uint32_t kYFloats = 2 * BM * BN;      // y accumulators of the tile: [plane][token][output]
-constexpr uint32_t kSmemBytes = STAGES * kStageBytes + kYFloats * 4 + 1024 /*align*/ + 256 /*barriers*/;
+constexpr uint32_t kSmemBytes = kYOff + kYFloats * 4 + 1024 /*align*/ + 512 /*barriers*/;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAcol = 2 * BM;              // A stage s at columns kAcol + 32 s
 constexpr uint32_t kIdesc = umma_idesc_bf16(2 * BN, 2 * BM);
@@ -100,6 +108,8 @@ struct Smem {
   uint64_t full_tma[STAGES];
   uint64_t full_a[STAGES];
   uint64_t empty[STAGES];
+  uint64_t full_c[CSTAGES];
+  uint64_t empty_c[CSTAGES];
   uint64_t acc_full;
   uint64_t acc_empty;
   uint64_t drain;
@@ -189,8 +199,8 @@ template <int kCap>
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ GemmParams<kCap> p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* ys = reinterpret_cast<float*>(smem + STAGES * kStageBytes);
-  Smem* S = reinterpret_cast<Smem*>(smem + STAGES * kStageBytes + kYFloats * 4);
+  float* ys = reinterpret_cast<float*>(smem + kYOff);
+  Smem* S = reinterpret_cast<Smem*>(smem + kYOff + kYFloats * 4);
   volatile int* abort = &S->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -198,13 +208,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   const int64_t t_first = blockIdx.x, t_step = gridDim.x;
 
   auto xtile = [&](int s) { return smem + s * kStageBytes; };  // X_re, then X_im 16 KB later
-  auto ctile = [&](int s) { return smem + s * kStageBytes + 2 * kTileX; };
+  auto ctile = [&](int c) { return smem + kCodeOff + c * kTileC; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&S->full_tma[s], 1);
       mbar_init(&S->full_a[s], kExpWarps);
       mbar_init(&S->empty[s], 1);
+    }
+    for (int c = 0; c < CSTAGES; ++c) {
+      mbar_init(&S->full_c[c], 1);
+      mbar_init(&S->empty_c[c], kExpWarps);
     }
     mbar_init(&S->acc_full, 1);
     mbar_init(&S->acc_empty, kEpiWarps);
@@ -241,8 +255,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         const int KB = (int)(L.K / BK), np = P * L.nbranch;
         bool ok = true;
         for (int q = 0; q < np && ok; ++q) {
-          const int t = q / L.nbranch, br = q % L.nbranch;
-          const int32_t crow = (int32_t)((int64_t)t * L.N + tl.n0);
           for (int kb = 0; kb < KB; ++kb, ++it) {
             const int s = it % STAGES;
             const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -253,7 +265,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             mbar_arrive_expect_tx(&S->full_tma[s], kTmaBytes);
             tma_load_2d(xtile(s), &L.tmap_x[0], kb * BK, (int32_t)tl.m0, &S->full_tma[s]);
             tma_load_2d(xtile(s) + kTileX, &L.tmap_x[1], kb * BK, (int32_t)tl.m0, &S->full_tma[s]);
-            tma_load_2d(ctile(s), &L.tmap_codes[br], kb * (BK / 4), crow, &S->full_tma[s]);
             ++issued[s];
           }
         }
@@ -306,6 +317,40 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       umma_commit(&S->drain);
       mbar_wait_bounded(&S->drain, 0u, &never);
     }
+  } else if (warp == kCodeWarp) {
+    // ------------------------------------------------------------ code producer: the 1 KB code tiles, up
+    // to CSTAGES stages ahead of the expanders (the activation stages are far fewer)
+    if (lane == 0) {
+      int issued[CSTAGES];
+      for (int c = 0; c < CSTAGES; ++c) issued[c] = 0;
+      int it = 0;
+      bool ok = true;
+      for (int64_t tt = t_first; tt < p.tiles && ok && !*abort; tt += t_step) {
+        const Tile tl = decode_tile(p, tt);
+        const GemmLayer& L = p.L[tl.li];
+        const int KB = (int)(L.K / BK), np = P * L.nbranch;
+        for (int q = 0; q < np && ok; ++q) {
+          const int t = q / L.nbranch, br = q % L.nbranch;
+          const int32_t crow = (int32_t)((int64_t)t * L.N + tl.n0);
+          for (int kb = 0; kb < KB; ++kb, ++it) {
+            const int c = it % CSTAGES;
+            const uint32_t ph = (uint32_t)(it / CSTAGES) & 1u;
+            if (!mbar_wait_bounded_ns(&S->empty_c[c], ph ^ 1u, abort, p.wait_ns)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&S->full_c[c], kTileC);
+            tma_load_2d(ctile(c), &L.tmap_codes[br], kb * (BK / 4), crow, &S->full_c[c]);
+            ++issued[c];
+          }
+        }
+      }
+      if (*abort) {
+        volatile int never = 0;
+        for (int c = 0; c < CSTAGES; ++c)
+          if (issued[c] > 0) mbar_wait_bounded(&S->full_c[c], (uint32_t)(issued[c] - 1) & 1u, &never);
+      }
+    }
   } else if (warp < kExpWarps) {
     // ------------------------------------------------------------ expanders
     const bool imag = lane >= 16;
@@ -319,20 +364,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       const int KB = (int)(L.K / BK), np = P * L.nbranch;
       for (int q = 0; q < np && ok; ++q) {
         for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          const int s = it % STAGES, cs = it % CSTAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u, cph = (uint32_t)(it / CSTAGES) & 1u;
           int w_ok = 1;
+          // the A stage is free once the MMAs that read it are done; the codes were loaded far ahead
           if (lane == 0)
-            w_ok = mbar_wait_bounded_ns(&S->empty[s], ph ^ 1u, abort, p.wait_ns) &&
-                   mbar_wait_bounded_ns(&S->full_tma[s], ph, abort, p.wait_ns);
+            w_ok = mbar_wait_bounded_ns(&S->full_c[cs], cph, abort, p.wait_ns) &&
+                   mbar_wait_bounded_ns(&S->empty[s], ph ^ 1u, abort, p.wait_ns);
           ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0;
           if (!ok) break;
           // Rows past N carry other stages' or no codes; their outputs are never stored.
-          const uint4 cw = *reinterpret_cast<const uint4*>(ctile(s) + o * 16);
+          const uint4 cw = *reinterpret_cast<const uint4*>(ctile(cs) + o * 16);
           const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
           uint32_t col[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) col[c] = expand_pair((w[c >> 3] >> (4 * (c & 7))) & 0xFu, imag);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S->empty_c[cs]);  // every lane has its code word in registers
           tmem_st_32x32b_x32(trow + 32 * s, col);
           tmem_wait_st();
           tc_fence_before();
@@ -371,6 +419,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           tmem_ld_32x32b_x32(trow + 32 * c, u);         // this lane's class, real plane, tokens 32c..
           tmem_ld_32x32b_x32(trow + BM + 32 * c, v);    // imaginary plane
           tmem_wait_ld();
+          if (c + 2 >= BM / 32) {
+            // this warp's last read of the accumulator: the next pass may overwrite it while the
+            // values in registers are applied
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S->acc_empty);
+          }
           // lane j < 16 (Br) takes tokens 32c + 0..15, lane j >= 16 (Bi) tokens 32c + 16..31;
           // each gets the other class's values of its tokens from lane j ^ 16.  The first pass of a
           // tile writes this lane's y entries, the later ones read, update and write them back.
@@ -402,9 +457,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             yim[i * BN] = cim[i];
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S->acc_empty);
       }
       // The tile's y is complete in shared memory.  Every epilogue warp takes the same decision to go
       // on (a lost wait anywhere stops them all at this point), then they store y together.
