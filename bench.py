@@ -233,7 +233,8 @@ class Block:
         """Our kernels per step (the L2-flush memset is not counted): conversion, quantizer (a stage
         kernel and a reduction kernel per stage), GEMV, GEMM."""
         gemv = 2  # activation digits (prep) + product
-        return len(self.cfg.layers) + 2 * self.T + gemv + len(self.gemm_layers)
+        gemm = 1  # one persistent launch over all layers
+        return len(self.cfg.layers) + 2 * self.T + gemv + gemm
 
 
 def oracle_sample_layers(rows_per_layer):
