@@ -37,7 +37,8 @@
 //   13    TMEM allocator and single-thread MMA issuer (M=128, N=256, K=16 per instruction)
 //   14    TMA producer of the codes: 64 x 16-byte tiles in a ring of 16 stages of their own, so
 //         that an expander finds its codes in place as soon as its A stage is free
-// TMEM: the accumulator (256 columns) and 4 stages of A (32 columns each).
+// TMEM: the accumulator (256 columns) and 8 stages of A (32 columns each), twice the activation
+// stages, so that the expanders run up to 8 stages ahead of the MMAs.
 // Every mbarrier wait is bounded; a lost wait sets IFQ_DEV_TIMEOUT, the CTA
 // drains its outstanding copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -53,7 +54,8 @@ namespace {
 constexpr int BM = 128;      // tokens per tile; the MMA's N is 2 BM (both planes)
 constexpr int BN = 64;       // outputs per tile; the MMA's M is 2 BN (Br and Bi rows)
 constexpr int BK = 64;       // K per stage (one 128-byte swizzle row of bf16)
-constexpr int STAGES = 4;                    // activation stages in shared memory = A stages in TMEM
+constexpr int STAGES = 4;                    // activation stages in shared memory
+constexpr int ASTAGES = 8;                   // stages of the expanded codes (A) in TMEM
 constexpr int CSTAGES = 16;                  // code stages: a ring of its own, filled far ahead
 constexpr int kExpWarps = 4;
 constexpr int kEpiWarps = 8;                 // two per TMEM lane quarter, each half the tokens
@@ -71,9 +73,9 @@ constexpr uint32_t kYFloats = 2 * BM * BN;      // y accumulators of the tile: [
 constexpr uint32_t kSmemBytes = kYOff + kYFloats * 4 + 1024 /*align*/ + 512 /*barriers*/;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAcol = 2 * BM;              // A stage s at columns kAcol + 32 s
+constexpr uint32_t kAcol = 2 * BM;              // A stage a at columns kAcol + 32 a
 constexpr uint32_t kIdesc = umma_idesc_bf16(2 * BN, 2 * BM);
-static_assert(kAcol + STAGES * (BK / 2) <= kTmemCols, "TMEM budget");
+static_assert(kAcol + ASTAGES * (BK / 2) <= kTmemCols, "TMEM budget");
 
 // One layer of a grouped call.  Its output tiles are numbered from tile_begin: token tile
 // (128 tokens) major, output tile (64 outputs) minor, so that the tiles running at the same time
@@ -106,8 +108,9 @@ static_assert(sizeof(GemmParams<IFQ_MAX_GROUP>) <= 32764, "kernel parameter bloc
 
 struct Smem {
   uint64_t full_tma[STAGES];
-  uint64_t full_a[STAGES];
   uint64_t empty[STAGES];
+  uint64_t full_a[ASTAGES];
+  uint64_t empty_a[ASTAGES];
   uint64_t full_c[CSTAGES];
   uint64_t empty_c[CSTAGES];
   uint64_t acc_full;
@@ -117,6 +120,8 @@ struct Smem {
   int abort;
   int epi_stop;
 };
+
+static_assert(sizeof(Smem) <= 512, "barrier block");
 
 struct Tile {
   int li;
@@ -213,8 +218,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&S->full_tma[s], 1);
-      mbar_init(&S->full_a[s], kExpWarps);
       mbar_init(&S->empty[s], 1);
+    }
+    for (int a = 0; a < ASTAGES; ++a) {
+      mbar_init(&S->full_a[a], kExpWarps);
+      mbar_init(&S->empty_a[a], 1);
     }
     for (int c = 0; c < CSTAGES; ++c) {
       mbar_init(&S->full_c[c], 1);
@@ -294,19 +302,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         if (!ok) break;
         tc_fence_after();
         for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          const int s = it % STAGES, sa = it % ASTAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u, pha = (uint32_t)(it / ASTAGES) & 1u;
           if (lane == 0)
             w_ok = mbar_wait_bounded_ns(&S->full_tma[s], ph, abort, p.wait_ns) &&
-                   mbar_wait_bounded_ns(&S->full_a[s], ph, abort, p.wait_ns);
+                   mbar_wait_bounded_ns(&S->full_a[sa], pha, abort, p.wait_ns);
           ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0;
           if (!ok) break;
           tc_fence_after();
           // the four K16 steps of the stage: B advances 32 bytes (2 descriptor units) per step inside the
           // 128-byte swizzle row, A 8 TMEM columns
-          umma_bf16_ta_x4(tmem, tmem + kAcol + 32 * s, xdesc0 + (uint64_t)((uint32_t)s * (kStageBytes >> 4)), kIdesc,
+          umma_bf16_ta_x4(tmem, tmem + kAcol + 32 * sa, xdesc0 + (uint64_t)((uint32_t)s * (kStageBytes >> 4)), kIdesc,
                           kb != 0);
-          umma_commit_elect(&S->empty[s]);
+          umma_commit_elect(&S->empty[s]);     // the activation stage may be refilled
+          umma_commit_elect(&S->empty_a[sa]);  // the A stage may be rewritten
         }
         if (!ok) break;
         umma_commit_elect(&S->acc_full);
@@ -364,13 +373,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       const int KB = (int)(L.K / BK), np = P * L.nbranch;
       for (int q = 0; q < np && ok; ++q) {
         for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % STAGES, cs = it % CSTAGES;
-          const uint32_t ph = (uint32_t)(it / STAGES) & 1u, cph = (uint32_t)(it / CSTAGES) & 1u;
+          const int sa = it % ASTAGES, cs = it % CSTAGES;
+          const uint32_t pha = (uint32_t)(it / ASTAGES) & 1u, cph = (uint32_t)(it / CSTAGES) & 1u;
           int w_ok = 1;
           // the A stage is free once the MMAs that read it are done; the codes were loaded far ahead
           if (lane == 0)
             w_ok = mbar_wait_bounded_ns(&S->full_c[cs], cph, abort, p.wait_ns) &&
-                   mbar_wait_bounded_ns(&S->empty[s], ph ^ 1u, abort, p.wait_ns);
+                   mbar_wait_bounded_ns(&S->empty_a[sa], pha ^ 1u, abort, p.wait_ns);
           ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0;
           if (!ok) break;
           // Rows past N carry other stages' or no codes; their outputs are never stored.
@@ -381,11 +390,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           for (int c = 0; c < 32; ++c) col[c] = expand_pair((w[c >> 3] >> (4 * (c & 7))) & 0xFu, imag);
           __syncwarp();
           if (lane == 0) mbar_arrive(&S->empty_c[cs]);  // every lane has its code word in registers
-          tmem_st_32x32b_x32(trow + 32 * s, col);
+          tmem_st_32x32b_x32(trow + 32 * sa, col);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&S->full_a[s]);
+          if (lane == 0) mbar_arrive(&S->full_a[sa]);
         }
       }
     }
