@@ -302,6 +302,11 @@ ifq_status ifq_dequantize(const ifq_dqtensor* tensors, int count, int T, ifq_str
  *                       then needs no workspace)
  *   x_re, x_im          [rows][K] bf16 bit patterns, device, 16-byte aligned
  *   y_re, y_im          [rows][N] float32, device, overwritten
+ *                       ("device" means an address the GPU can use: x and y may
+ *                       also be pinned host memory in the unified address space,
+ *                       which the kernels then read and write over PCIe; for
+ *                       ifq_gemv at B <= 2 x is read once, by the preparation
+ *                       kernel, so that costs little)
  *   rot_re, rot_im      optional epilogue rotation, both NULL = none: when set,
  *                       output [r][n] is multiplied by the complex number
  *                       rot_re[r][n] + i rot_im[r][n] ([rows][N] float32,
