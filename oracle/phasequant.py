@@ -71,7 +71,7 @@ def phase_code(a, b):
       k = 1  iff  b > |a|   or (a = b and b > 0)
       k = 2  iff -a > |b|   or (b = -a and a < 0)
       k = 3  iff -b > |a|   or (a = b and b < 0)
-    and w = 0 gives k = 0.  No rounding enters, so this is the judged form.
+    and w = 0 gives k = 0.  No rounding enters, so this is the form the parity checks use.
     """
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)
