@@ -476,3 +476,44 @@ def test_products_of_every_width_the_quantizer_accepts(K):
         assert int(st.item()) == 0
         check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), cun, sun, cwn, swn,
                       W.bf16_to_f32_numpy(xr), W.bf16_to_f32_numpy(xi))
+
+
+def test_grouped_call_of_more_than_eight_layers():
+    """20 layers in one call (the 32-layer parameter block) of mixed shapes, with and without the
+    conj branch: every layer's decode (B = 1, 2, 5) and prefill (M = 131) outputs within the bound of
+    the oracle, and the grouped prefill equal to one call per layer bit for bit (a GEMM output is summed
+    in a fixed order, whatever the tile schedule)."""
+    rng = np.random.default_rng(2020)
+    T = 2
+    shapes = [(N, K, conj) for N, K in ((16, 64), (37, 128), (64, 320), (130, 192), (80, 64)) for conj in (True, False)]
+    shapes = (shapes * 2)[:20]
+    quant = []
+    for N, K, conj in shapes:
+        ws = [_rand_complex(rng, N, K)] + ([_rand_complex(rng, N, K, 0.03)] if conj else [])
+        outs = gpu_quantize([(to_dev(a), to_dev(b)) for a, b in ws], T)
+        quant.append(outs)
+    host = [[(c.cpu().numpy(), s.cpu().numpy()) for c, s in outs] for outs in quant]
+    for rows, is_gemm in ((1, False), (2, False), (5, False), (131, True)):
+        descs, xs = [], []
+        for (N, K, conj), outs in zip(shapes, quant):
+            xr = torch.from_numpy(rng.standard_normal((rows, K)).astype(np.float32)).to(torch.bfloat16)
+            xi = torch.from_numpy(rng.standard_normal((rows, K)).astype(np.float32)).to(torch.bfloat16)
+            cw, sw = (outs[1][0], outs[1][1]) if conj else (None, None)
+            descs.append(layer_desc(outs[0][0], outs[0][1], cw, sw, xr.to(DEV), xi.to(DEV), N, K, rows))
+            xs.append((xr, xi))
+        if is_gemm:
+            Q.ifq_gemm(descs, T, rows)
+        else:
+            run_gemv(descs, T, rows)
+        torch.cuda.synchronize()
+        for (N, K, conj), h, d, (xr, xi) in zip(shapes, host, descs, xs):
+            cw, sw = (h[1][0], h[1][1]) if conj else (None, None)
+            check_product(d["y_re"].cpu().numpy(), d["y_im"].cpu().numpy(), h[0][0], h[0][1], cw, sw,
+                          W.bf16_to_f32_numpy(xr), W.bf16_to_f32_numpy(xi))
+        if is_gemm:
+            for d in descs:
+                single = dict(d, y_re=torch.empty_like(d["y_re"]), y_im=torch.empty_like(d["y_im"]))
+                Q.ifq_gemm([single], T, rows)
+                torch.cuda.synchronize()
+                assert torch.equal(single["y_re"].view(torch.int32), d["y_re"].view(torch.int32))
+                assert torch.equal(single["y_im"].view(torch.int32), d["y_im"].view(torch.int32))
