@@ -712,6 +712,13 @@ def e2e_decode(block, steps, warmup):
                                 "copies_only_ms": t_copies_only * 1e3}}
 
 
+def bench_config(ws, B, M, T):
+    """The workload of a bench line; both arms report the same one."""
+    return {"workload": WORKLOAD, "decode_batch": B, "prefill_M": M, "stages": T,
+            "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+            "l2": "256 MiB L2 flush before the GEMV in every step; conversion/quantizer inputs (1.6 GB) exceed L2"}
+
+
 def max_over_ranks(values, device):
     """Element-wise max of every rank's values (times in seconds); a no-op on one rank."""
     t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
@@ -850,10 +857,7 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16 activations x 2-bit codes, f32 accumulate; f64 scale reduction",
         "data": "synthetic: seeded N(0,0.02) real weights, N(0,1) bf16 activations",
-        "config": {"workload": WORKLOAD, "decode_batch": block.B, "prefill_M": block.M, "stages": block.T,
-                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
-                   "l2": "256 MiB L2 flush before the GEMV in every step; conversion/quantizer inputs (1.6 GB) "
-                         "exceed L2"},
+        "config": bench_config(ws, block.B, block.M, block.T),
         "prefill_gemm": {"value": job_rate(ws, block.gemm_flops(), t_gemm) / 1e12, "unit": "TOP/s (equivalent dense, 8 M N K per stage and branch)",
                          "frac_of_burst_bf16": gemm_tops / tf_burst, "frac_of_sustained_bf16": gemm_tops / tf_sus},
         "roofline": {"kernel": dominant, "bound": rl["bound"], "achieved": rl["achieved"], "peak": rl["peak"],
@@ -898,7 +902,7 @@ def run_reference(args):
     line = {"metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": WORKLOAD, "decode_batch": 1, "stages": 2},
+            "config": bench_config(ws, 1, 2048, 2),
             "cpu_baseline": cpu,
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
