@@ -1,5 +1,7 @@
-// Decode product for one token (B = 1) on the integer tensor cores, exactly
+// Decode product for one or two tokens (B = 1, 2) on the integer tensor cores, exactly
 // ("Fairy2i write-up" §2.1, §4.2; "iFairy article" §二.2; "iFairy talk notes" §2.3.1).
+// The description below is the one-token case; two tokens share each operand's extraction
+// (half_chunk_mma) and keep one int32 sum per (plane, token).
 //
 // Re-coding the 2-bit code.  With k = 2 s + c (c: axis bit, s: sign bit), the
 // real and imaginary parts of the codeword [1, i, -1, -i][k] are
