@@ -145,3 +145,35 @@ def test_misaligned_shards_are_refused():
     s[0]["w_re"] = s[0]["w_re"][:-1]
     with pytest.raises(ValueError):
         shard.quantize_row_split(s, T, 0, 2, stage=np_stage, finish=np_finish, gather=lambda l, z: [l, l])
+
+
+def _gather_main(rank, world, port, q):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from bit_complex_quantized_b200.shard import gather_rows, row_shards
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        N, K, rows = 1100, 200, 3
+        full = torch.arange(rows * N, dtype=torch.float32).reshape(rows, N)
+        n0, n1 = row_shards(N, K, world)[rank]
+        got = gather_rows(full[:, n0:n1].contiguous(), N, rank, world, K)
+        q.put((rank, bool(torch.equal(got, full))))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gather_rows_reassembles_the_outputs_of_a_row_split():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_gather_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=240) for _ in procs)
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    assert res == {0: True, 1: True}
